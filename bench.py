@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layout -> FP8 dispatch -> BF16 combine path on B200.
+
+One step = cgl_get_layout + cgl_dispatch_fp8 + cgl_combine over one batch of
+synthetic routing (the 4096-token prefill shape by default: hidden 7168, 256
+experts in 8 groups, top-4 groups / top-8 experts, 64 logical ranks) with all
+inputs resident in HBM.  The metric is the step's algorithmic HBM bytes per
+second; per-kernel microseconds and fractions of the measured HBM peak are in
+the same JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (weak
+scaling, no data-path collective); the timing is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from combine_get_layout_02_b200 import workloads as W  # noqa: E402
+
+METRIC = "dispatch+combine µs and HBM GB/s (% of peak) at 4096 tok×7168, top-8/256"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM bytes per launch read by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the kernels at the 4096-token prefill shape, with the sha256 of the kernel
+# source they were taken on; a changed source reports traffic null.
+NCU_TRAFFIC = {}
+
+
+def _src_sha(name: str) -> str:
+    p = os.path.join(ROOT, "combine_get_layout_02_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(kernel: str, src: str):
+    rec = NCU_TRAFFIC.get(kernel)
+    if not rec or rec.get("src_sha") != _src_sha(src):
+        return None
+    return rec["bytes"]
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- distributed
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(backend: str, timeout_s: float = 120.0):
+    import datetime
+
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity with one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each replica draws its own batch of the same workload."""
+    return seed + 1000 * rank
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- steps
+
+def workload_label(wl: W.Workload) -> str:
+    return f"{wl.name}: {wl.description}"
+
+
+class GpuStep:
+    """Device buffers for one workload and the launch sequence of one step."""
+
+    def __init__(self, wl: W.Workload, seed: int, device):
+        import torch
+
+        import combine_get_layout_02_b200 as cgl
+
+        self.cgl, self.torch, self.wl, self.dev = cgl, torch, wl, device
+        inp = W.make_inputs(wl, seed)
+        n, h, k = wl.num_tokens, wl.hidden, wl.topk
+        self.host = inp
+        self.M = n * k
+        y_host = W.expert_outputs(self.M, h, seed)
+        self.host_y = y_host
+
+        def bf16(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+
+        self.x = bf16(inp.x).to(device)
+        self.idx = torch.from_numpy(inp.topk_idx).to(device)
+        self.w = torch.from_numpy(inp.topk_w).to(device)
+        self.y = bf16(y_host).to(device)
+        self.grad = bf16(inp.grad).to(device) if inp.grad is not None else None
+        self.status = cgl.new_status(device)
+        E, R = wl.num_experts, wl.num_ranks
+        self.ws = torch.empty(cgl.layout_workspace_bytes(n, k, E, R), dtype=torch.uint8, device=device)
+        self.cap = 0
+        if wl.padded:   # padded receive buffers: size them from a first compact call (host reads max)
+            lay = cgl.get_layout(self.idx, E, R, 0, workspace=self.ws, status=self.status)
+            self.cap = int(lay.max_count.item())
+        self.lay = cgl.get_layout(self.idx, E, R, self.cap, workspace=self.ws, status=self.status)
+        rows = self.lay.num_recv_rows
+        self.rows = rows
+        if wl.fp8:
+            self.recv_x = torch.empty((rows, h), dtype=torch.uint8, device=device)
+            self.recv_scale = torch.empty((rows, h // 128), dtype=torch.float32, device=device)
+            if wl.padded:   # y rows follow the padded layout
+                self.y = self.y.new_zeros((rows, h))
+                self.y[self.lay.dst_pos.flatten().long()] = bf16(y_host).to(device)
+        else:
+            self.recv_x = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
+            self.grad_recv = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((n, h), dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize(device)
+        self.bytes = W.algorithmic_bytes(wl)
+
+    def kernels(self):
+        """(name, launches per step, algorithmic bytes per launch) of each step phase."""
+        b = self.bytes
+        ph = [("layout", 2, b["layout"])]
+        if self.wl.fp8:
+            ph.append(("dispatch_fp8", 1, b["dispatch_fp8"]))
+        else:
+            ph.append(("dispatch_bf16", 1, b["dispatch_bf16"]))
+        ph.append(("combine", 1, b["combine"]))
+        if self.wl.with_grad:
+            ph.append(("combine_backward", 1, b["dispatch_bf16"]))
+        return ph
+
+    def step_bytes(self):
+        return sum(v for _, _, v in self.kernels())
+
+    def run(self, events=None):
+        """One step; if `events` is a list, record an event after each phase."""
+        cgl, wl = self.cgl, self.wl
+        E, R = wl.num_experts, wl.num_ranks
+        rec = (lambda: events.append(self._event())) if events is not None else (lambda: None)
+        rec()
+        cgl.get_layout(self.idx, E, R, self.cap, workspace=self.ws, out=self.lay, status=self.status)
+        rec()
+        if wl.fp8:
+            cgl.dispatch_fp8(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
+                             recv_scale=self.recv_scale, status=self.status)
+        else:
+            cgl.dispatch_bf16(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
+                              status=self.status)
+        rec()
+        cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
+        rec()
+        if wl.with_grad:
+            cgl.dispatch_bf16(self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv,
+                              status=self.status)
+            rec()
+
+    def _event(self):
+        e = self.torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+
+def run_e2e(step: GpuStep, steps: int):
+    """Same step through the public API with host buffers: pinned H2D of the
+    step's inputs, the kernels, D2H of the combined output and the counts."""
+    import torch
+
+    wl = step.wl
+    pin = lambda t: t.cpu().pin_memory()
+    hx, hidx, hw, hy = pin(step.x), pin(step.idx), pin(step.w), pin(step.y)
+    hg = pin(step.grad) if step.grad is not None else None
+    hout = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    htpe = torch.empty(step.lay.tokens_per_expert.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hidx, hw, hy) + ((hg,) if hg is not None else ()))
+    d2h = hout.numel() * hout.element_size() + htpe.numel() * 4
+
+    def one():
+        step.x.copy_(hx, non_blocking=True)
+        step.idx.copy_(hidx, non_blocking=True)
+        step.w.copy_(hw, non_blocking=True)
+        step.y.copy_(hy, non_blocking=True)
+        if hg is not None:
+            step.grad.copy_(hg, non_blocking=True)
+        step.run()
+        htpe.copy_(step.lay.tokens_per_expert, non_blocking=True)
+        hout.copy_(step.out, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+
+def oracle_step_seconds(inp: W.Inputs, y: np.ndarray, tokens: int, reps_min_s: float, max_reps: int):
+    """Time the oracle's layout + dispatch + combine on the first `tokens` tokens."""
+    import oracle
+
+    wl = inp.workload
+    idx = inp.topk_idx[:tokens]
+    x = inp.x[:tokens]
+    w = inp.topk_w[:tokens]
+    reps, t_total = 0, 0.0
+    while reps < max_reps and (reps == 0 or t_total < reps_min_s):
+        t0 = time.perf_counter()
+        L = oracle.get_layout(idx, wl.num_experts, wl.num_ranks, 0)
+        rows = idx.size
+        if wl.fp8:
+            oracle.dispatch_fp8(x, L.dst_pos, rows)
+        else:
+            oracle.dispatch_bf16(x, L.dst_pos, rows)
+        oracle.combine(y[:rows], L.dst_pos, w)
+        if wl.with_grad:
+            oracle.dispatch_bf16(inp.grad[:tokens], L.dst_pos, rows)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    return t_total, reps
+
+
+def step_bytes_for(wl: W.Workload, tokens: int) -> int:
+    b = W.algorithmic_bytes(wl, tokens)
+    tot = b["layout"] + b["combine"] + (b["dispatch_fp8"] if wl.fp8 else b["dispatch_bf16"])
+    if wl.with_grad:
+        tot += b["dispatch_bf16"]
+    return tot
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- arms
+
+def base_line(args, wl, n_gpus):
+    return {
+        "metric": METRIC, "unit": "GB/s", "n_gpus": n_gpus, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": workload_label(wl), "num_tokens": wl.num_tokens, "hidden": wl.hidden,
+            "num_experts": wl.num_experts, "num_groups": wl.num_groups, "topk_group": wl.topk_group,
+            "topk": wl.topk, "num_ranks": wl.num_ranks,
+            "storage": ("x bf16 -> e4m3 rows + f32 1x128 scales; combine bf16 in, f32 accumulate, bf16 out"
+                        if wl.fp8 else "x bf16 rows; combine bf16; combine-backward bf16 rows"),
+            "parallelism": f"replicas x{n_gpus} (logical EP ranks inside each GPU)",
+            "l2": "no flush: inputs larger than L2 (each step touches "
+                  f"{step_bytes_for(wl, wl.num_tokens) / 1e9:.2f} GB)",
+            "seed": args.seed,
+        },
+    }
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    wl = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(wl, args.seed)
+    y = W.expert_outputs(inp.topk_idx.size, wl.hidden, args.seed)
+    threads = oracle.set_threads(cpu_threads())
+    # size the per-step sample so that warmup + steps end within ~2 minutes
+    t_full, _ = oracle_step_seconds(inp, y, wl.num_tokens, 0.0, 1)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    tokens = wl.num_tokens if t_full <= budget else max(16, int(wl.num_tokens * budget / t_full) // 16 * 16)
+    for _ in range(args.warmup):
+        oracle_step_seconds(inp, y, tokens, 0.0, 1)
+    times = []
+    for _ in range(args.steps):
+        t, _ = oracle_step_seconds(inp, y, tokens, 0.0, 1)
+        times.append(t)
+    sec = sum(times) / len(times)
+    gbs = step_bytes_for(wl, tokens) / sec / 1e9
+    line = base_line(args, wl, world)
+    sample = (f"first {tokens} of {wl.num_tokens} tokens per step (layout + "
+              f"{'dispatch_fp8' if wl.fp8 else 'dispatch_bf16'} + combine), C oracle, OpenMP over tokens")
+    line.update({
+        "impl": "reference", "value": gbs, "ms_per_step": sec * 1e3,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    })
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    wl = W.WORKLOADS[args.workload]
+    step = GpuStep(wl, rank_seed(args.seed, rank), dev)
+    phases = step.kernels()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)   # let nvidia-smi start sampling before the timed region
+    evs = []
+    for _ in range(args.steps):
+        ev = []
+        step.run(ev)
+        evs.append(ev)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per_phase = [0.0] * len(phases)
+    for ev in evs:
+        for i in range(len(phases)):
+            per_phase[i] += ev[i].elapsed_time(ev[i + 1])
+    per_phase = [v / args.steps for v in per_phase]
+    ms = total_ms / args.steps
+    red = max_over_ranks([ms] + per_phase, device=dev)
+    ms, per_phase = red[0], red[1:]
+    status_bits = step.cgl.status_bits(step.status)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = run_e2e(step, args.e2e_steps)
+        e2e_ms = max_over_ranks([e2e_ms], device=dev)[0]
+        e2e = {"value": step.step_bytes() * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        barrier()
+        return 0
+    peak, peak_src = hbm_peak()
+    kernels = {}
+    for (name, launches, nbytes), t in zip(phases, per_phase):
+        gbs = nbytes / (t * 1e-3) / 1e9
+        kernels[name] = {"us": t * 1e3, "launches_per_step": launches, "bytes": nbytes,
+                         "gbs": gbs, "frac_of_peak": gbs / peak}
+    dom = max(phases, key=lambda p: p[2])[0]
+    src = {"combine": "combine.cu", "dispatch_fp8": "dispatch.cu", "dispatch_bf16": "dispatch.cu",
+           "layout": "layout.cu", "combine_backward": "dispatch.cu"}[dom]
+    roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
+            "bytes_per_launch": kernels[dom]["bytes"]}
+    line = base_line(args, wl, world)
+    value = step.step_bytes() * world / (ms * 1e-3) / 1e9
+    line.update({
+        "value": value, "ms_per_step": ms, "roofline": roof, "kernels": kernels,
+        "dispatch_plus_combine_us": sum(kernels[n]["us"] for n in kernels if n != "layout"),
+        "gpu_launches": args.steps * sum(p[1] for p in phases),
+        "clocks": clocks, "device_status": status_bits or "ok",
+    })
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+
+        threads = oracle.set_threads(cpu_threads())
+        t, reps = oracle_step_seconds(step.host, step.host_y, wl.num_tokens, args.cpu_seconds, 1000)
+        gbs = step_bytes_for(wl, wl.num_tokens) * reps / t / 1e9
+        line["cpu_baseline"] = {
+            "value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} full {wl.num_tokens}-token steps (same inputs), {t:.1f} s, C oracle with OpenMP over tokens"}
+    print(json.dumps(line), flush=True)
+    barrier()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=W.WORKLOAD_ORDER, default="prefill")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    try:
+        return run_ours(args)
+    finally:
+        import torch.distributed as dist
+
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,182 @@
+// The exported C ABI (declared in include/cgl.h): argument checks, then one
+// call into the launchers.  Host-visible errors return before any launch.
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace cgl {
+
+namespace {
+
+std::mutex g_mu;
+
+struct KernelCache {
+    const void *kernel;
+    int device;
+    size_t smem;         // dynamic shared memory limit set so far
+    int ctas_per_sm;     // occupancy at kThreads, 0 = not computed
+};
+std::vector<KernelCache> g_kernels;
+int g_sms[256] = {0};
+
+KernelCache &entry(const void *kernel, int device) {
+    for (auto &e : g_kernels)
+        if (e.kernel == kernel && e.device == device) return e;
+    g_kernels.push_back({kernel, device, 48 * 1024, 0});
+    return g_kernels.back();
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int opt_sms(const cgl_opts *o) { return o ? o->num_sms : 0; }
+int opt_cap(const cgl_opts *o) { return o ? o->capacity : 0; }
+
+}  // namespace
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 0;
+    if (g_sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_sms[dev] = v;
+    }
+    return g_sms[dev];
+}
+
+bool ensure_smem_attr(const void *kernel, size_t bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    KernelCache &e = entry(kernel, dev);
+    if (bytes <= e.smem) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return false;
+    e.smem = bytes;
+    return true;
+}
+
+int copy_grid(const void *kernel, int threads, int64_t work_ctas, int num_sms_cap) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const int sms = device_sm_count();
+    if (sms <= 0) return 0;
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        KernelCache &e = entry(kernel, dev);
+        if (e.ctas_per_sm == 0) {
+            int v = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, threads, 0) != cudaSuccess)
+                return 0;
+            e.ctas_per_sm = v > 0 ? v : 1;
+        }
+        per_sm = e.ctas_per_sm;
+    }
+    const int use_sms = (num_sms_cap > 0 && num_sms_cap < sms) ? num_sms_cap : sms;
+    const int64_t cap = (int64_t)use_sms * per_sm;
+    return (int)(work_ctas < cap ? work_ctas : cap);
+}
+
+}  // namespace cgl
+
+using namespace cgl;
+
+extern "C" {
+
+int cgl_version(void) { return 100; }
+
+const char *cgl_status_string(int s) {
+    switch (s) {
+        case CGL_OK: return "ok";
+        case CGL_EINVAL: return "invalid argument";
+        case CGL_EALIGN: return "misaligned pointer";
+        case CGL_ERANGE: return "expert id or receive row out of range";
+        case CGL_ECAPACITY: return "padded expert capacity exceeded";
+        case CGL_ETIMEOUT: return "bounded wait timed out";
+        case CGL_ECUDA: return "CUDA runtime error";
+        case CGL_ENOTIMPL: return "not implemented";
+        default: return "unknown status";
+    }
+}
+
+static bool layout_sizes_ok(int64_t n, int k, int E, int R) {
+    return n >= 0 && k >= 1 && k <= kMaxTopk && E >= 1 && E <= kMaxExperts && R >= 1 && R <= E &&
+           E % R == 0 && n * (int64_t)k < ((int64_t)1 << 31);
+}
+
+size_t cgl_layout_workspace_bytes(int64_t n, int k, int E, int R) {
+    if (!layout_sizes_ok(n, k, E, R)) return 0;
+    return layout_workspace_bytes(n, E, R);
+}
+
+cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t n, int k, int E, int R,
+                          const cgl_opts *opts, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                          uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
+                          int32_t *dst_pos, int32_t *recv_src, void *workspace,
+                          size_t workspace_bytes, uint32_t *status_dev, void *stream) {
+    if (!layout_sizes_ok(n, k, E, R)) return CGL_EINVAL;
+    const int cap = opt_cap(opts);
+    if (cap < 0 || (int64_t)E * cap >= ((int64_t)1 << 31)) return CGL_EINVAL;
+    const int64_t rows = cap > 0 ? (int64_t)E * cap : n * k;
+    if (!tokens_per_expert || !tokens_per_rank || !expert_offset || !max_count || !workspace)
+        return CGL_EINVAL;
+    if (n > 0 && (!topk_idx || !dst_pos || !is_token_in_rank)) return CGL_EINVAL;
+    if (rows > 0 && !recv_src) return CGL_EINVAL;
+    if (workspace_bytes < layout_workspace_bytes(n, E, R)) return CGL_EINVAL;
+    if (!aligned(topk_idx, 4) || !aligned(tokens_per_expert, 4) || !aligned(tokens_per_rank, 4) ||
+        !aligned(expert_offset, 4) || !aligned(max_count, 4) || !aligned(dst_pos, 4) ||
+        !aligned(recv_src, 4) || !aligned(status_dev, 4) || !aligned(is_token_in_rank, 16) ||
+        !aligned(workspace, 16))
+        return CGL_EALIGN;
+    return launch_layout(topk_idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank,
+                         is_token_in_rank, expert_offset, max_count, dst_pos, recv_src, workspace,
+                         status_dev, static_cast<cudaStream_t>(stream));
+}
+
+cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
+                            uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
+                            const cgl_opts *opts, uint32_t *status_dev, void *stream) {
+    if (n < 0 || h <= 0 || h % 128 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0)
+        return CGL_EINVAL;
+    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
+    if (n > 0 && recv_rows > 0 && (!recv_x || !recv_scale)) return CGL_EINVAL;
+    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) ||
+        !aligned(recv_scale, 4) || !aligned(status_dev, 4))
+        return CGL_EALIGN;
+    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, opt_sms(opts),
+                               status_dev, static_cast<cudaStream_t>(stream));
+}
+
+cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
+                             uint16_t *recv_x, int64_t recv_rows, const cgl_opts *opts,
+                             uint32_t *status_dev, void *stream) {
+    if (n < 0 || h <= 0 || h % 8 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
+    if (n > 0 && recv_rows > 0 && !recv_x) return CGL_EINVAL;
+    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) || !aligned(status_dev, 4))
+        return CGL_EALIGN;
+    return launch_dispatch_bf16(x, n, h, k, dst_pos, recv_x, recv_rows, opt_sms(opts), status_dev,
+                                static_cast<cudaStream_t>(stream));
+}
+
+cgl_status cgl_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_pos,
+                       const float *topk_weights, int64_t n, int h, int k, uint16_t *out,
+                       const cgl_opts *opts, uint32_t *status_dev, void *stream) {
+    if (n < 0 || h <= 0 || h % 8 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (n > 0 && (!dst_pos || !topk_weights || !out)) return CGL_EINVAL;
+    if (n > 0 && recv_rows > 0 && !y) return CGL_EINVAL;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(dst_pos, 4) ||
+        !aligned(topk_weights, 4) || !aligned(status_dev, 4))
+        return CGL_EALIGN;
+    return launch_combine(y, recv_rows, dst_pos, topk_weights, n, h, k, out, opt_sms(opts),
+                          status_dev, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

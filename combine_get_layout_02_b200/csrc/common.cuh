@@ -1,0 +1,58 @@
+// Device helpers shared by the layout, dispatch and combine kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "cgl.h"
+
+namespace cgl {
+
+constexpr uint32_t kErrRange = 1u << CGL_ERANGE;
+constexpr uint32_t kErrCapacity = 1u << CGL_ECAPACITY;
+
+constexpr int kMaxTopk = 32;
+constexpr int kMaxExperts = 1024;
+
+// OR an error bit into the caller's status word (error paths only).
+__device__ __forceinline__ void report(uint32_t *status, uint32_t bit) {
+    if (status != nullptr) atomicOr(status, bit);
+}
+
+// 16-byte global load through the non-coherent path, not kept in L1: every
+// byte the copy kernels read is read once.
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// 16-byte global store with the streaming (evict-first) cache hint.
+__device__ __forceinline__ void st_cs_v4(void *p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Two floats -> two E4M3 bytes, round to nearest even, finite values past 448
+// clamp to +-448 (PTX cvt ... satfinite).  `lo` lands in bits 7:0.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two floats -> two BF16 values, round to nearest even.  `lo` lands in bits 15:0.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Widen the low / high BF16 of a 32-bit word to float (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+}  // namespace cgl

@@ -1,0 +1,183 @@
+/*
+ * cgl.h -- C ABI of the single-GPU MoE layout / dispatch / combine library
+ * (libcgl.so, CUDA kernels for B200, sm_100a).
+ *
+ * What the calls compute.  The DeepEP pages describe all-to-all GPU kernels
+ * for MoE "dispatch" (send each token to the experts its gate picked) and
+ * "combine" (merge the experts' outputs back, accumulating), FP8 dispatch and
+ * BF16 combine, group-limited gating ("top-4 groups, top-8 experts"), and a
+ * host that waits for a GPU-produced receive count:
+ *   - "DeepEP ... CPO" GitHub-issue mirror, section "Technical Overview of DeepEP";
+ *   - 智东西 news article (yunnanlong.com), the feature list and "具体性能方面";
+ *   - brainleap.ai "【Day2】DeepEP", sections "DeepEP是什么", "All-to-All通信"
+ *     (combine accumulates) and the caption "CPU 将隐式地等待 GPU 接收到的计数信号";
+ *   - flashmla.org/de "DeepEP", the feature and benchmark-setting paragraphs.
+ * Here the expert-parallel ranks are logical partitions of ONE GPU: rank r owns
+ * experts [r*E/R, (r+1)*E/R), every "send" is a row copy inside this GPU's
+ * memory, and there is no collective.
+ *
+ * Conventions for every call.
+ *   - Pointers named as device buffers are device (or managed) memory that the
+ *     CALLER allocates and frees; the library allocates nothing and keeps no
+ *     pointer after a call returns.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and is asynchronous: outputs are ready when the stream is.
+ *   - Arrays are dense and row-major.  BF16 values are passed as their 16-bit
+ *     patterns (uint16_t); FP8 values as E4M3 ("fn": no infinities, max 448)
+ *     bytes.
+ *   - Errors the host can see (sizes, null or misaligned pointers) are returned
+ *     at once and nothing is launched.  Errors only the GPU can see are OR-ed
+ *     into `*status_dev` as bits (1u << CGL_ERANGE, 1u << CGL_ECAPACITY, ...);
+ *     the caller zeroes that word and reads it after synchronising.
+ *     `status_dev` may be NULL, in which case those errors go unreported (the
+ *     kernels still skip the offending copies).  No kernel traps or asserts.
+ *   - Calls that share output buffers must not overlap on the GPU.
+ *   - Limits: num_topk in [1, 32]; num_experts in [1, 1024];
+ *     num_tokens * num_topk < 2^31; num_experts % num_ranks == 0.
+ */
+#ifndef CGL_H
+#define CGL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum cgl_status {
+    CGL_OK = 0,
+    CGL_EINVAL = 1,     /* bad size or argument, or a required pointer is NULL */
+    CGL_EALIGN = 2,     /* a pointer is not aligned as the call requires */
+    CGL_ERANGE = 3,     /* (device) an expert id < -1 or >= E, or a receive row outside the buffer */
+    CGL_ECAPACITY = 4,  /* (device) a padded expert received more copies than its capacity */
+    CGL_ETIMEOUT = 5,   /* (device) a bounded wait gave up; reserved, no current kernel waits */
+    CGL_ECUDA = 6,      /* the CUDA runtime refused a launch or an attribute call */
+    CGL_ENOTIMPL = 7    /* not implemented */
+} cgl_status;
+
+/* Per-call options.  A NULL options pointer means all fields zero. */
+typedef struct cgl_opts {
+    /* Cap the grid of the copy kernels to this many SMs' worth of CTAs
+     * (0 = all SMs).  This is the SM-count control the DeepEP pages list for
+     * their normal kernels (news article feature list; flashmla.org/de). */
+    int32_t num_sms;
+    /* cgl_get_layout only.  0: compact receive rows, expert e's copies at rows
+     * [expert_offset[e], expert_offset[e+1]).  > 0: padded receive buffers of
+     * `capacity` rows per expert, expert e's copies at rows [e*capacity, ...);
+     * the decode setting pads to the largest per-expert count, which the host
+     * reads from a first, compact call (max_count). */
+    int32_t capacity;
+} cgl_opts;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int cgl_version(void);
+
+/* A static string naming a cgl_status value (or "unknown status"). */
+const char *cgl_status_string(int status);
+
+/*
+ * Bytes of device workspace cgl_get_layout needs for these sizes (per-block
+ * histograms).  Host-only; returns 0 for invalid sizes.
+ */
+size_t cgl_layout_workspace_bytes(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
+
+/*
+ * cgl_get_layout -- the dispatch layout: how many copies each expert and each
+ * logical rank receives, where they start, and the receive row of every
+ * (token, slot) copy.  Pages: the dispatch described under "DeepEP是什么" and
+ * "All-to-All通信" (brainleap "Day2 DeepEP"), whose receive counts the host
+ * waits on (caption "CPU 将隐式地等待 GPU 接收到的计数信号").
+ *
+ * In (device):
+ *   topk_idx          int32 [num_tokens, num_topk]; expert id per slot, -1 = no copy.
+ * Out (device, all written in full by the call):
+ *   tokens_per_expert int32 [E]: copies routed to expert e (including copies
+ *                     dropped for capacity).
+ *   tokens_per_rank   int32 [R]: distinct tokens with at least one copy on rank r.
+ *   is_token_in_rank  uint8 [num_tokens, R]: 1 if token t has a copy on rank r, else 0.
+ *   expert_offset     int32 [E + 1]: exclusive prefix sum of tokens_per_expert
+ *                     (expert order, so each rank's experts are contiguous).
+ *   max_count         int32 [1]: max over e of tokens_per_expert.
+ *   dst_pos           int32 [num_tokens, num_topk]: receive row of the copy, -1
+ *                     when the slot is masked, out of range or over capacity.
+ *   recv_src          int32 [num_tokens*num_topk] (compact) or [E*capacity]
+ *                     (padded): t*num_topk + j of the copy in each receive row,
+ *                     -1 for rows that receive nothing.
+ * Order: inside each expert, copies are in ascending token order (ascending
+ * slot for a repeated expert within one token), i.e. a stable counting sort.
+ * workspace: device, >= cgl_layout_workspace_bytes(...) bytes, 16-byte aligned,
+ *   any contents; it is scratch for the call and may be reused afterwards.
+ * Device errors: CGL_ERANGE for ids < -1 or >= E (those slots make no copy),
+ *   CGL_ECAPACITY when a padded expert overflows (late copies dropped).
+ * Host errors: CGL_EINVAL (sizes, NULL outputs, small workspace), CGL_EALIGN
+ *   (int32 arrays not 4-byte aligned, workspace or is_token_in_rank not 16-byte aligned).
+ */
+cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_topk,
+                          int num_experts, int num_ranks, const cgl_opts *opts,
+                          int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                          uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
+                          int32_t *dst_pos, int32_t *recv_src, void *workspace,
+                          size_t workspace_bytes, uint32_t *status_dev, void *stream);
+
+/*
+ * cgl_dispatch_fp8 -- FP8 dispatch: quantise each token once and write its
+ * copies to the receive rows.  Pages: "FP8 dispatch, BF16 combine" in the
+ * benchmark settings (news article "具体性能方面"; brainleap "DeepEP 的性能表现";
+ * flashmla.org/de) and "原生FP8 调度支持" (brainleap key techniques, item 5).
+ *
+ * For token t and each block b of 128 consecutive hidden values:
+ *   amax = max |x|, amax_c = max(amax, 1e-4), scale = amax_c / 448,
+ *   inv = 448 / amax_c (IEEE binary32 divisions), q = e4m3_rn_satfinite(x * inv);
+ * then for every slot j with dst_pos[t, j] = row >= 0:
+ *   recv_x[row, :] = q, recv_scale[row, b] = scale.
+ * In (device): x BF16 [num_tokens, hidden]; dst_pos int32 [num_tokens, num_topk]
+ *   (from cgl_get_layout).
+ * Out (device): recv_x uint8 [num_recv_rows, hidden], recv_scale fp32
+ *   [num_recv_rows, hidden/128].  Rows that receive no copy are NOT written.
+ * Requires hidden % 128 == 0; x and recv_x 16-byte aligned; dst_pos and
+ * recv_scale 4-byte aligned.
+ * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows (that copy is skipped).
+ */
+cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t num_tokens, int hidden, int num_topk,
+                            const int32_t *dst_pos, uint8_t *recv_x, float *recv_scale,
+                            int64_t num_recv_rows, const cgl_opts *opts, uint32_t *status_dev,
+                            void *stream);
+
+/*
+ * cgl_dispatch_bf16 -- BF16 dispatch: recv_x[dst_pos[t, j], :] = x[t, :] bit for
+ * bit.  The same call re-dispatches gradient rows by a forward layout
+ * (combine-backward, unweighted).  Pages: dispatch as above; BF16 is the
+ * combine format of the benchmark settings.
+ * In (device): x BF16 [num_tokens, hidden]; dst_pos int32 [num_tokens, num_topk].
+ * Out (device): recv_x BF16 [num_recv_rows, hidden]; rows with no copy are not written.
+ * Requires hidden % 8 == 0; x and recv_x 16-byte aligned.
+ * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows.
+ */
+cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t num_tokens, int hidden, int num_topk,
+                             const int32_t *dst_pos, uint16_t *recv_x, int64_t num_recv_rows,
+                             const cgl_opts *opts, uint32_t *status_dev, void *stream);
+
+/*
+ * cgl_combine -- BF16 combine: gather each token's expert outputs back and
+ * reduce them with the top-k weights.  Pages: combine "accumulates"
+ * (brainleap "All-to-All通信", the combine bullet), BF16 combine (benchmark
+ * settings).
+ *   out[t, h] = bf16_rn( ((+0 + w[t,0]*y0) + w[t,1]*y1) + ... ), y_j = y[dst_pos[t, j], h],
+ * each product and each sum one binary32 operation (no fused multiply-add),
+ * slots in order j = 0..k-1, slots with dst_pos < 0 skipped.
+ * In (device): y BF16 [num_recv_rows, hidden]; dst_pos int32 [num_tokens, num_topk];
+ *   topk_weights fp32 [num_tokens, num_topk] (used as given).
+ * Out (device): out BF16 [num_tokens, hidden], every element written.
+ * Requires hidden % 8 == 0; y and out 16-byte aligned.
+ * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows (that slot is skipped).
+ */
+cgl_status cgl_combine(const uint16_t *y, int64_t num_recv_rows, const int32_t *dst_pos,
+                       const float *topk_weights, int64_t num_tokens, int hidden, int num_topk,
+                       uint16_t *out, const cgl_opts *opts, uint32_t *status_dev, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CGL_H */

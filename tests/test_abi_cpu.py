@@ -1,0 +1,113 @@
+"""The C ABI on a machine without a GPU: libcgl.so loads, exports every function
+include/cgl.h declares, and rejects bad arguments on the host before launching
+anything (no call here reaches the GPU)."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import combine_get_layout_02_b200 as cgl
+from combine_get_layout_02_b200 import build as cbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    cbuild.build()
+    return cgl.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "cgl.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(cgl_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("cgl_get_layout", "cgl_dispatch_fp8", "cgl_dispatch_bf16", "cgl_combine",
+                 "cgl_layout_workspace_bytes", "cgl_status_string", "cgl_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version(L):
+    assert L.cgl_version() >= 100
+    assert L.cgl_status_string(0) == b"ok"
+    assert L.cgl_status_string(cgl.ECAPACITY) != L.cgl_status_string(cgl.ERANGE)
+    assert L.cgl_status_string(99) == b"unknown status"
+
+
+def test_workspace_size_rules(L):
+    assert L.cgl_layout_workspace_bytes(4096, 8, 256, 64) > 0
+    assert L.cgl_layout_workspace_bytes(0, 8, 256, 64) > 0          # empty batch still needs one block
+    assert L.cgl_layout_workspace_bytes(4096, 8, 256, 60) == 0      # E % R != 0
+    assert L.cgl_layout_workspace_bytes(4096, 33, 256, 64) == 0     # k > 32
+    assert L.cgl_layout_workspace_bytes(4096, 8, 2048, 64) == 0     # E > 1024
+    assert L.cgl_layout_workspace_bytes(-1, 8, 256, 64) == 0
+    assert L.cgl_layout_workspace_bytes(2 ** 28, 8, 256, 64) == 0   # N*k >= 2^31
+
+
+FAKE = 0x10000  # 64 KiB-aligned, never dereferenced: every call below fails its host checks
+
+
+def _opts(cap=0, sms=0):
+    return C.byref(cgl.Opts(sms, cap))
+
+
+def test_get_layout_host_errors(L):
+    p = FAKE
+    ws = L.cgl_layout_workspace_bytes(128, 8, 256, 64)
+    args = lambda **kw: dict(dict(idx=p, n=128, k=8, E=256, R=64, opts=_opts(), tpe=p, tpr=p, itr=p,
+                                  off=p, mx=p, dst=p, src=p, ws=p, wsb=ws, st=p, stream=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.cgl_get_layout(a["idx"], a["n"], a["k"], a["E"], a["R"], a["opts"], a["tpe"],
+                                a["tpr"], a["itr"], a["off"], a["mx"], a["dst"], a["src"], a["ws"],
+                                a["wsb"], a["st"], a["stream"])
+
+    assert call(R=60) == cgl.EINVAL
+    assert call(k=0) == cgl.EINVAL
+    assert call(wsb=ws - 1) == cgl.EINVAL
+    assert call(dst=None) == cgl.EINVAL
+    assert call(opts=_opts(cap=-1)) == cgl.EINVAL
+    assert call(tpe=None) == cgl.EINVAL
+    assert call(dst=p + 2) == cgl.EALIGN
+    assert call(itr=p + 4) == cgl.EALIGN
+    assert call(ws=p + 8) == cgl.EALIGN
+
+
+def test_copy_kernels_host_errors(L):
+    p = FAKE
+    # FP8 dispatch needs H % 128 == 0 and 16-byte aligned rows
+    assert L.cgl_dispatch_fp8(p, 16, 7000, 8, p, p, p, 128, None, None, None) == cgl.EINVAL
+    assert L.cgl_dispatch_fp8(p, 16, 7168, 0, p, p, p, 128, None, None, None) == cgl.EINVAL
+    assert L.cgl_dispatch_fp8(p + 8, 16, 7168, 8, p, p, p, 128, None, None, None) == cgl.EALIGN
+    assert L.cgl_dispatch_fp8(p, 16, 7168, 8, p, p + 4, p, 128, None, None, None) == cgl.EALIGN
+    assert L.cgl_dispatch_fp8(p, 16, 7168, 8, None, p, p, 128, None, None, None) == cgl.EINVAL
+    assert L.cgl_dispatch_fp8(p, 16, 7168, 8, p, p, p, 128, _opts(sms=-1), None, None) == cgl.EINVAL
+    # BF16 dispatch: H % 8
+    assert L.cgl_dispatch_bf16(p, 16, 7164, 8, p, p, 128, None, None, None) == cgl.EINVAL
+    assert L.cgl_dispatch_bf16(p, 16, 7168, 8, p, p + 2, 128, None, None, None) == cgl.EALIGN
+    # combine
+    assert L.cgl_combine(p, 128, p, p, 16, 7168, 33, p, None, None, None) == cgl.EINVAL
+    assert L.cgl_combine(p, -1, p, p, 16, 7168, 8, p, None, None, None) == cgl.EINVAL
+    assert L.cgl_combine(p, 128, p, None, 16, 7168, 8, p, None, None, None) == cgl.EINVAL
+    assert L.cgl_combine(p, 128, p, p, 16, 7168, 8, p + 8, None, None, None) == cgl.EALIGN
+    assert L.cgl_combine(p, 128, p, p + 1, 16, 7168, 8, p, None, None, None) == cgl.EALIGN
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    with pytest.raises(TypeError):
+        cgl.combine(torch.zeros(8, 8, dtype=torch.bfloat16), torch.zeros(1, 8, dtype=torch.int32),
+                    torch.zeros(1, 8))

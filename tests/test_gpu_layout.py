@@ -1,0 +1,101 @@
+"""GPU layout (cgl_get_layout) against the oracle, bit for bit, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import combine_get_layout_02_b200 as cgl
+from combine_get_layout_02_b200 import workloads as W
+
+from helpers import dev, i32
+
+pytestmark = pytest.mark.gpu
+
+
+def run_both(oracle_mod, idx, E, R, cap=0):
+    st = cgl.new_status(dev())
+    lay = cgl.get_layout(i32(idx), E, R, cap, status=st)
+    torch.cuda.synchronize()
+    ref = oracle_mod.get_layout(idx, E, R, cap)
+    got = {f: getattr(lay, f).cpu().numpy() for f in
+           ("tokens_per_expert", "tokens_per_rank", "is_token_in_rank", "expert_offset", "dst_pos", "recv_src")}
+    for f, g in got.items():
+        r = getattr(ref, f)
+        assert g.shape == r.shape, f
+        assert np.array_equal(g, r), f"{f} differs at {np.argwhere(g != r)[:5].tolist()}"
+    assert int(lay.max_count.item()) == ref.max_count
+    bits = int(st.item())
+    assert bool(bits & (1 << cgl.ERANGE)) == bool(ref.flags & oracle_mod.FLAG_RANGE)
+    assert bool(bits & (1 << cgl.ECAPACITY)) == bool(ref.flags & oracle_mod.FLAG_CAPACITY)
+    return lay, ref
+
+
+@pytest.mark.parametrize("name", W.WORKLOAD_ORDER)
+def test_layout_full_size_workloads(oracle_mod, name):
+    inp = W.make_inputs(name, 0)
+    wl = inp.workload
+    lay, ref = run_both(oracle_mod, inp.topk_idx, wl.num_experts, wl.num_ranks, 0)
+    if wl.padded:
+        run_both(oracle_mod, inp.topk_idx, wl.num_experts, wl.num_ranks, int(lay.max_count.item()))
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_layout_random_ragged(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    E = int(rng.choice([8, 16, 64, 256, 1024]))
+    R = int(rng.choice([r for r in (1, 2, 4, 8, 32, 64, E) if E % r == 0]))
+    k = int(rng.choice([1, 2, 3, 4, 6, 8, 13, 32]))
+    n = int(rng.choice([1, 7, 255, 256, 257, 1000, 3333]))
+    if k <= E:
+        idx = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    else:
+        idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    idx[rng.random((n, k)) < 0.05] = -1
+    run_both(oracle_mod, idx, E, R, 0)
+
+
+def test_layout_duplicates_bad_ids_and_overflow(oracle_mod):
+    rng = np.random.default_rng(42)
+    n, k, E, R = 700, 8, 16, 4
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)          # duplicates within tokens
+    bad = rng.random((n, k)) < 0.02
+    idx[bad] = rng.choice([-5, -2, E, E + 100], bad.sum())
+    idx[rng.random((n, k)) < 0.05] = -1
+    run_both(oracle_mod, idx, E, R, 0)
+    run_both(oracle_mod, idx, E, R, 300)      # padded, no overflow
+    run_both(oracle_mod, idx, E, R, 200)      # padded, some experts overflow
+
+
+def test_layout_skewed_hot_expert(oracle_mod):
+    # one expert takes every token: the worst case for same-expert contention
+    n, k, E, R = 5000, 4, 64, 8
+    rng = np.random.default_rng(1)
+    idx = np.stack([np.concatenate([[3], rng.permutation(np.delete(np.arange(E), 3))[:k - 1]])
+                    for _ in range(n)]).astype(np.int32)
+    run_both(oracle_mod, idx, E, R, 0)
+
+
+def test_layout_empty_and_all_masked(oracle_mod):
+    run_both(oracle_mod, np.zeros((0, 8), np.int32), 256, 64, 0)
+    run_both(oracle_mod, np.zeros((0, 8), np.int32), 256, 64, 4)
+    run_both(oracle_mod, np.full((300, 8), -1, np.int32), 256, 64, 0)
+
+
+def test_layout_max_sizes(oracle_mod):
+    rng = np.random.default_rng(9)
+    n, k, E = 2048, 32, 1024
+    idx = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    run_both(oracle_mod, idx, E, 1024, 0)
+    run_both(oracle_mod, idx, E, 1, 0)
+
+
+def test_layout_repeated_calls_reuse_workspace(oracle_mod):
+    inp = W.make_inputs("prefill", 3)
+    wl = inp.workload
+    ws = torch.full((cgl.layout_workspace_bytes(4096, 8, 256, 64),), 0x5A, dtype=torch.uint8, device=dev())
+    idx = i32(inp.topk_idx)
+    a = cgl.get_layout(idx, 256, 64, workspace=ws)
+    b = cgl.get_layout(idx, 256, 64, workspace=ws)
+    assert torch.equal(a.dst_pos, b.dst_pos)
+    ref = oracle_mod.get_layout(inp.topk_idx, 256, 64)
+    assert np.array_equal(b.dst_pos.cpu().numpy(), ref.dst_pos)
