@@ -21,6 +21,9 @@ int copy_grid(const void *kernel, int threads, int64_t work_ctas, int num_sms_ca
 
 size_t layout_workspace_bytes(int64_t n, int E, int R);
 
+// Dynamic shared memory of the layout assign kernel per block (bytes).
+size_t layout_assign_smem_bytes(int E, int k);
+
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                          int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
                          int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,

@@ -268,6 +268,10 @@ layout_assign_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, i
 
 size_t layout_workspace_bytes(int64_t n, int E, int R) { return ws_layout(n, E, R).bytes; }
 
+size_t layout_assign_smem_bytes(int E, int k) {
+    return (size_t)(3 * E + kWarps * E + kTokensPerBlock * k) * sizeof(int32_t);
+}
+
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                          int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
                          int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,

@@ -120,6 +120,45 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
                           int32_t *dst_pos, int32_t *recv_src, void *workspace,
                           size_t workspace_bytes, uint32_t *status_dev, void *stream);
 
+/* Size of the device scratch array behind cgl_get_layout_noalloc. */
+#define CGL_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/*
+ * cgl_get_layout_noalloc -- cgl_get_layout for callers that cannot allocate
+ * device memory.  The pages have no counterpart of this entry point.
+ *
+ * Who needs it: hosts that give the library only pre-planned input and output
+ * buffers and own all other device memory (engine plugins, serving runtimes
+ * with a fixed memory plan), callers that must not take the device-wide
+ * synchronisation that cudaFree implies, and callers that reach only this C
+ * ABI without a CUDA allocator.  They cannot provide the workspace that
+ * cgl_get_layout takes.
+ *
+ * Same arguments, outputs, ordering and errors as cgl_get_layout, minus the
+ * workspace: the scratch is a fixed device array of CGL_NOALLOC_SCRATCH_BYTES
+ * (256 KiB) inside libcgl.so, held by every GPU that loads the library until
+ * the process exits.  The call allocates nothing (no cudaMalloc or cudaFree,
+ * no allocating library routine); the caller still passes every input and
+ * output buffer.
+ * Limits, rejected with CGL_EINVAL before anything is launched:
+ *   cgl_layout_workspace_bytes(...) <= CGL_NOALLOC_SCRATCH_BYTES
+ *     (at E = 256, R = 64: up to 52,224 tokens), and
+ *   11 * num_experts + 256 * num_topk <= 12288 (the layout kernels then fit in
+ *     the default 48 KiB of shared memory per block; any num_topk at E <= 372).
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once and caches it; make that first call before any
+ * stream capture.  CGL_ECUDA if the lookup fails.
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents (nothing in it needs to start at zero).  Calls whose work overlaps
+ * on the GPU race on it: serialise them (one stream per device, or events).
+ */
+cgl_status cgl_get_layout_noalloc(const int32_t *topk_idx, int64_t num_tokens, int num_topk,
+                                  int num_experts, int num_ranks, const cgl_opts *opts,
+                                  int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                                  uint8_t *is_token_in_rank, int32_t *expert_offset,
+                                  int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
+                                  uint32_t *status_dev, void *stream);
+
 /*
  * cgl_dispatch_fp8 -- FP8 dispatch: quantise each token once and write its
  * copies to the receive rows.  Pages: "FP8 dispatch, BF16 combine" in the

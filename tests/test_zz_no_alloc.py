@@ -1,0 +1,96 @@
+"""cgl_get_layout_noalloc through the C ABI: same results as cgl_get_layout.
+
+This entry point is for callers that cannot allocate device memory (hosts that
+pass only pre-planned input/output buffers, callers that must avoid the
+synchronisation of cudaFree, C-only callers without a CUDA allocator); its
+scratch is a fixed device array inside libcgl.so, shared by all calls.  The
+test runs two calls in a row on different inputs, so that the second sees
+whatever the first left in that array, and compares each with cgl_get_layout
+(the existing entry point, with a caller-allocated workspace) bit for bit, the
+tolerance for integer outputs.  It also checks that sizes past the array's
+limit are refused before any launch.  The file sorts last so that a run that
+stops at the first failure has already run everything else.
+"""
+
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+import combine_get_layout_02_b200 as cgl
+from combine_get_layout_02_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+FIELDS = ("tokens_per_expert", "tokens_per_rank", "is_token_in_rank", "expert_offset", "max_count",
+          "dst_pos", "recv_src")
+
+
+def _fn():
+    f = cgl.lib().cgl_get_layout_noalloc
+    P, I64, I = C.c_void_p, C.c_int64, C.c_int
+    f.argtypes = [P, I64, I, I, I, C.POINTER(cgl.Opts), P, P, P, P, P, P, P, P, P]
+    f.restype = I
+    return f
+
+
+def _noalloc(idx: torch.Tensor, E: int, R: int, cap: int = 0):
+    n, k = idx.shape
+    dev = idx.device
+    rows = E * cap if cap > 0 else n * k
+    # poison every output so that a skipped write shows up
+    out = {
+        "tokens_per_expert": torch.full((E,), -7, dtype=torch.int32, device=dev),
+        "tokens_per_rank": torch.full((R,), -7, dtype=torch.int32, device=dev),
+        "is_token_in_rank": torch.full((n, R), 0xEE, dtype=torch.uint8, device=dev),
+        "expert_offset": torch.full((E + 1,), -7, dtype=torch.int32, device=dev),
+        "max_count": torch.full((1,), -7, dtype=torch.int32, device=dev),
+        "dst_pos": torch.full((n, k), -7, dtype=torch.int32, device=dev),
+        "recv_src": torch.full((rows,), -7, dtype=torch.int32, device=dev),
+    }
+    st = cgl.new_status(dev)
+    code = _fn()(idx.data_ptr(), n, k, E, R, C.byref(cgl.Opts(0, cap)),
+                 *[out[f].data_ptr() for f in FIELDS], st.data_ptr(),
+                 torch.cuda.current_stream().cuda_stream)
+    assert code == cgl.OK, cgl.lib().cgl_status_string(code)
+    return out, st
+
+
+def _reference(idx: torch.Tensor, E: int, R: int, cap: int = 0):
+    st = cgl.new_status(idx.device)
+    lay = cgl.get_layout(idx, E, R, cap, status=st)
+    return {f: getattr(lay, f) for f in FIELDS}, st
+
+
+def test_noalloc_matches_get_layout_on_two_calls_in_a_row():
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cases = []
+    a = W.make_inputs("skewed", 0)          # 16384 tokens: the larger scratch footprint first
+    cases.append((torch.from_numpy(a.topk_idx).to(dev), 256, 64, 0))
+    b = W.make_inputs("decode", 0)          # then a small padded layout over the leftovers
+    idx_b = torch.from_numpy(b.topk_idx).to(dev)
+    cap = int(_reference(idx_b, 256, 32)[0]["max_count"].item())
+    cases.append((idx_b, 256, 32, cap))
+    for idx, E, R, c in cases:
+        got, st = _noalloc(idx, E, R, c)
+        ref, st_ref = _reference(idx, E, R, c)
+        torch.cuda.synchronize()
+        for f in FIELDS:
+            assert torch.equal(got[f], ref[f]), f
+        assert int(st.item()) == int(st_ref.item()) == 0
+
+
+def test_noalloc_refuses_sizes_past_its_scratch():
+    dev = torch.device("cuda", 0)
+    fake = 1 << 16   # never dereferenced: the size check comes first
+    f = _fn()
+    args = [fake] * 7
+    # 60000 tokens at E=256, R=64 need more than the 256 KiB scratch array
+    assert cgl.layout_workspace_bytes(60000, 8, 256, 64) > 256 * 1024
+    assert f(fake, 60000, 8, 256, 64, None, *args, None, None) == cgl.EINVAL
+    # E=1024 with k=8 would need more than 48 KiB of shared memory per block
+    assert f(fake, 100, 8, 1024, 64, None, *args, None, None) == cgl.EINVAL
+    # within the limits the same fake pointers are only refused for alignment
+    assert f(fake + 2, 100, 8, 256, 64, None, *args, None, None) == cgl.EALIGN
