@@ -11,7 +11,9 @@
 // flight per thread), then accumulates acc = acc + w_j * y_j with separate
 // round-to-nearest multiply and add (no contraction to FMA), j ascending,
 // and stores one 16-byte BF16 vector.  A warp reads 512 contiguous bytes of
-// each of the token's k rows and writes 512 contiguous output bytes.
+// each of the token's k rows and writes 512 contiguous output bytes.  The
+// launch uses programmatic dependent launch (blocks wait in griddepcontrol
+// before their first global read).
 #include "common.cuh"
 #include "launch.h"
 
@@ -26,6 +28,8 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(const uint16_t *__restrict__ y, int64_t recv_rows,
                const int32_t *__restrict__ dst_pos, const float *__restrict__ w, int64_t n, int h,
                int k, uint16_t *__restrict__ out, uint32_t *status) {
+    griddep_launch_dependents();
+    griddep_wait();                   // y and dst_pos may come from the kernels just before
     const int chunks = h >> 3;
     const int64_t total = n * chunks;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -87,8 +91,9 @@ cgl_status launch_combine(const uint16_t *y, int64_t recv_rows, const int32_t *d
     const int grid = copy_grid((const void *)combine_kernel, kThreads,
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;
-    combine_kernel<<<grid, kThreads, 0, stream>>>(y, recv_rows, dst_pos, w, n, h, k, out, status);
-    return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    const cudaError_t err = launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, stream, y, recv_rows,
+                                       dst_pos, w, n, h, k, out, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 }  // namespace cgl

@@ -51,6 +51,16 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
     return r;
 }
 
+// Programmatic dependent launch (sm_90+).  launch_dependents lets the next
+// kernel in the stream, if it was launched with programmatic stream
+// serialisation, start its blocks early; wait blocks until every prerequisite
+// grid has completed and its memory operations are visible.  A kernel must not
+// read anything an earlier kernel may have written before it has waited.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Widen the low / high BF16 of a 32-bit word to float (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -13,7 +13,9 @@
 // and every store of a warp covers 512 contiguous bytes of one receive row.
 // For FP8 a 128-value scale block is 8 adjacent lanes; their absmax is
 // combined with three xor-shuffles.  The grid is a multiple of the resident
-// CTAs per SM and loops grid-stride.
+// CTAs per SM and loops grid-stride.  Launches use programmatic dependent
+// launch: blocks start while the layout kernels drain and wait (griddepcontrol)
+// before their first global read.
 #include "common.cuh"
 #include "launch.h"
 
@@ -27,6 +29,8 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                     const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
                     float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
+    griddep_launch_dependents();
+    griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4;        // 16 values per thread
     const int nblk = h >> 7;          // 128-value scale blocks per row
     const int64_t total = n * chunks; // a multiple of 8: scale groups never straddle
@@ -90,6 +94,8 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                      const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
                      int64_t recv_rows, uint32_t *status) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int chunks = h >> 3;        // 8 values per thread
     const int64_t total = n * chunks;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -119,9 +125,9 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
     const int grid = copy_grid((const void *)dispatch_fp8_kernel, kThreads,
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;
-    dispatch_fp8_kernel<<<grid, kThreads, 0, stream>>>(x, n, h, k, dst_pos, recv_x, recv_scale,
-                                                       recv_rows, status);
-    return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    const cudaError_t err = launch_pdl(dispatch_fp8_kernel, dim3(grid), dim3(kThreads), 0, stream, x, n, h,
+                                       k, dst_pos, recv_x, recv_scale, recv_rows, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
@@ -132,9 +138,9 @@ cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, cons
     const int grid = copy_grid((const void *)dispatch_bf16_kernel, kThreads,
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;
-    dispatch_bf16_kernel<<<grid, kThreads, 0, stream>>>(x, n, h, k, dst_pos, recv_x, recv_rows,
-                                                        status);
-    return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    const cudaError_t err = launch_pdl(dispatch_bf16_kernel, dim3(grid), dim3(kThreads), 0, stream, x, n,
+                                       h, k, dst_pos, recv_x, recv_rows, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 }  // namespace cgl

@@ -19,10 +19,30 @@ int device_sm_count();
 // (SMs in use) x (resident CTAs per SM).
 int copy_grid(const void *kernel, int threads, int64_t work_ctas, int num_sms_cap);
 
+// Launch `kernel` with programmatic stream serialisation: it may start while
+// the previous kernel in the stream is finishing, and must griddep_wait()
+// before reading anything that kernel (or an earlier one) wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 size_t layout_workspace_bytes(int64_t n, int E, int R);
 
-// Dynamic shared memory of the layout assign kernel per block (bytes).
-size_t layout_assign_smem_bytes(int E, int k);
+// True if some layout kernel for these sizes needs more shared memory than a
+// kernel gets without raising its attribute (host-side bookkeeping on first use).
+bool layout_needs_smem_optin(int E, int R, int k);
 
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                          int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,

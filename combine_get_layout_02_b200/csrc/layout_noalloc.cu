@@ -61,7 +61,7 @@ extern "C" cgl_status cgl_get_layout_noalloc(
     if (need == 0 || need > kScratchBytes) return CGL_EINVAL;
     // stay within the default 48 KiB of shared memory per block, so that no
     // launch here has to raise a kernel attribute first
-    if (cgl::layout_assign_smem_bytes(num_experts, num_topk) > 48 * 1024) return CGL_EINVAL;
+    if (cgl::layout_needs_smem_optin(num_experts, num_ranks, num_topk)) return CGL_EINVAL;
     void *scratch = scratch_on_current_device();
     if (scratch == nullptr) return CGL_ECUDA;
     return cgl_get_layout(topk_idx, num_tokens, num_topk, num_experts, num_ranks, opts,

@@ -51,7 +51,7 @@ typedef enum cgl_status {
     CGL_EALIGN = 2,     /* a pointer is not aligned as the call requires */
     CGL_ERANGE = 3,     /* (device) an expert id < -1 or >= E, or a receive row outside the buffer */
     CGL_ECAPACITY = 4,  /* (device) a padded expert received more copies than its capacity */
-    CGL_ETIMEOUT = 5,   /* (device) a bounded wait gave up; reserved, no current kernel waits */
+    CGL_ETIMEOUT = 5,   /* (device) a bounded wait between the layout's blocks gave up (~1 s) */
     CGL_ECUDA = 6,      /* the CUDA runtime refused a launch or an attribute call */
     CGL_ENOTIMPL = 7    /* not implemented */
 } cgl_status;
@@ -107,7 +107,8 @@ size_t cgl_layout_workspace_bytes(int64_t num_tokens, int num_topk, int num_expe
  * Order: inside each expert, copies are in ascending token order (ascending
  * slot for a repeated expert within one token), i.e. a stable counting sort.
  * workspace: device, >= cgl_layout_workspace_bytes(...) bytes, 16-byte aligned,
- *   any contents; it is scratch for the call and may be reused afterwards.
+ *   any contents; it is scratch for the call and may be reused afterwards
+ *   (calls that overlap on the GPU must not share one).
  * Device errors: CGL_ERANGE for ids < -1 or >= E (those slots make no copy),
  *   CGL_ECAPACITY when a padded expert overflows (late copies dropped).
  * Host errors: CGL_EINVAL (sizes, NULL outputs, small workspace), CGL_EALIGN
@@ -142,9 +143,11 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
  * output buffer.
  * Limits, rejected with CGL_EINVAL before anything is launched:
  *   cgl_layout_workspace_bytes(...) <= CGL_NOALLOC_SCRATCH_BYTES
- *     (at E = 256, R = 64: up to 52,224 tokens), and
- *   11 * num_experts + 256 * num_topk <= 12288 (the layout kernels then fit in
- *     the default 48 KiB of shared memory per block; any num_topk at E <= 372).
+ *     (at E = 256, R = 64: up to 51,968 tokens), and
+ *   256 * (num_topk | 1) + 12 * num_experts + num_ranks
+ *     + (num_ranks > 64 ? 256 * ceil(num_ranks / 32) : 0) <= 12032
+ *     (the layout kernels then fit in the default 48 KiB of shared memory per
+ *     block; with num_ranks <= 64: any num_topk up to E = 293, num_topk <= 8 up to E = 805).
  * Set-up: the first call on a device (with that device current) looks up the
  * array's device address once and caches it; make that first call before any
  * stream capture.  CGL_ECUDA if the lookup fails.

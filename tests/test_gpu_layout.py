@@ -99,3 +99,24 @@ def test_layout_repeated_calls_reuse_workspace(oracle_mod):
     assert torch.equal(a.dst_pos, b.dst_pos)
     ref = oracle_mod.get_layout(inp.topk_idx, 256, 64)
     assert np.array_equal(b.dst_pos.cpu().numpy(), ref.dst_pos)
+
+
+def test_layout_two_kernel_path_many_blocks(oracle_mod):
+    # more than 256 blocks of 256 tokens: the layout runs as two kernels
+    rng = np.random.default_rng(11)
+    n, k, E, R = 70000, 2, 64, 16
+    idx = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    idx[rng.random((n, k)) < 0.03] = -1
+    run_both(oracle_mod, idx, E, R, 0)
+    run_both(oracle_mod, idx, E, R, 2400)
+
+
+def test_layout_two_kernel_path_large_shared_memory_with_duplicates(oracle_mod):
+    # E = 1024, k = 32 needs more than 48 KiB of shared memory per block: two kernels;
+    # repeated experts inside tokens take the in-order walk
+    rng = np.random.default_rng(12)
+    n, k, E, R = 900, 32, 1024, 128
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    idx[:, 5] = idx[:, 3]                      # every token repeats one expert
+    run_both(oracle_mod, idx, E, R, 0)
+    run_both(oracle_mod, idx, E, R, 64)
