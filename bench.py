@@ -41,7 +41,11 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per launch read by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the kernels at the 4096-token prefill shape, with the sha256 of the kernel
 # source they were taken on; a changed source reports traffic null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "combine": {"bytes": 506999296, "src_sha": "b4d10dad3865f683"},
+    "dispatch_fp8": {"bytes": 242101248, "src_sha": "12e36f8c2e7dbd8e"},
+    "layout": {"bytes": 198400, "src_sha": "041e4a9928bdb3da"},
+}
 
 
 def _src_sha(name: str) -> str:
@@ -222,7 +226,9 @@ class GpuStep:
     def kernels(self):
         """(name, launches per step, algorithmic bytes per launch) of each step phase."""
         b = self.bytes
-        ph = [("layout", 2, b["layout"])]
+        wl = self.wl
+        nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_experts, wl.num_ranks)
+        ph = [("layout", nl, b["layout"])]
         if self.wl.fp8:
             ph.append(("dispatch_fp8", 1, b["dispatch_fp8"]))
         else:
@@ -422,23 +428,36 @@ def run_ours(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)   # let nvidia-smi start sampling before the timed region
+    # timed region: K steps, one event on each side, nothing between the kernels
+    # (an event between two kernels stops the next one from launching early)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    for _ in range(args.steps):
+        step.run()
+    e_end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    ms = e_start.elapsed_time(e_end) / args.steps
+
+    # per-kernel durations: a second pass of K steps with an event after every
+    # kernel; each duration includes the launch gap those events add
     evs = []
     for _ in range(args.steps):
         ev = []
         step.run(ev)
         evs.append(ev)
     torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
     barrier()
-    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
     per_phase = [0.0] * len(phases)
     for ev in evs:
         for i in range(len(phases)):
             per_phase[i] += ev[i].elapsed_time(ev[i + 1])
     per_phase = [v / args.steps for v in per_phase]
-    ms = total_ms / args.steps
-    red = max_over_ranks([ms] + per_phase, device=dev)
-    ms, per_phase = red[0], red[1:]
+    ms_instr = evs[0][0].elapsed_time(evs[-1][-1]) / args.steps
+    red = max_over_ranks([ms, ms_instr] + per_phase, device=dev)
+    ms, ms_instr, per_phase = red[0], red[1], red[2:]
     status_bits = step.cgl.status_bits(step.status)
 
     e2e = None
@@ -463,13 +482,17 @@ def run_ours(args):
     roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
-            "bytes_per_launch": kernels[dom]["bytes"]}
+            "bytes_per_launch": kernels[dom]["bytes"],
+            "timing": "CUDA events around each launch in the instrumented pass (launch gap included)"}
     line = base_line(args, wl, world)
     value = step.step_bytes() * world / (ms * 1e-3) / 1e9
     line.update({
         "value": value, "ms_per_step": ms, "roofline": roof, "kernels": kernels,
         "dispatch_plus_combine_us": sum(kernels[n]["us"] for n in kernels if n != "layout"),
         "gpu_launches": args.steps * sum(p[1] for p in phases),
+        "kernel_timing": ("per-kernel us from a second pass of the same K steps with a CUDA event "
+                          f"after every kernel ({ms_instr * 1e3:.1f} us/step there vs {ms * 1e3:.1f} clean); "
+                          "each includes the launch gap the events add"),
         "clocks": clocks, "device_status": status_bits or "ok",
     })
     if e2e:

@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "CglError", "Layout", "lib", "get_layout", "dispatch_fp8", "dispatch_bf16", "combine",
-    "layout_workspace_bytes", "status_bits", "check_status", "new_status",
+    "layout_workspace_bytes", "layout_kernel_count", "status_bits", "check_status", "new_status",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,8 @@ def lib():
         L.cgl_status_string.restype = C.c_char_p
         L.cgl_layout_workspace_bytes.argtypes = [I64, I, I, I]
         L.cgl_layout_workspace_bytes.restype = C.c_size_t
+        L.cgl_layout_kernel_count.argtypes = [I64, I, I, I]
+        L.cgl_layout_kernel_count.restype = I
         L.cgl_get_layout.argtypes = [P, I64, I, I, I, OP, P, P, P, P, P, P, P, P, C.c_size_t, P, P]
         L.cgl_get_layout.restype = I
         L.cgl_dispatch_fp8.argtypes = [P, I64, I, I, P, P, P, I64, OP, P, P]
@@ -140,6 +142,11 @@ def check_status(status: torch.Tensor, where: str = "device"):
 
 def layout_workspace_bytes(num_tokens: int, num_topk: int, num_experts: int, num_ranks: int) -> int:
     return int(lib().cgl_layout_workspace_bytes(num_tokens, num_topk, num_experts, num_ranks))
+
+
+def layout_kernel_count(num_tokens: int, num_topk: int, num_experts: int, num_ranks: int) -> int:
+    """Kernels one get_layout call launches for these sizes on the current device (1 or 2)."""
+    return int(lib().cgl_layout_kernel_count(num_tokens, num_topk, num_experts, num_ranks))
 
 
 class Layout(NamedTuple):

@@ -113,6 +113,11 @@ size_t cgl_layout_workspace_bytes(int64_t n, int k, int E, int R) {
     return layout_workspace_bytes(n, E, R);
 }
 
+int cgl_layout_kernel_count(int64_t n, int k, int E, int R) {
+    if (!layout_sizes_ok(n, k, E, R)) return -1;
+    return layout_fused_fits(n, k, E, R) ? 1 : 2;
+}
+
 cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t n, int k, int E, int R,
                           const cgl_opts *opts, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
                           uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,

@@ -6,16 +6,22 @@
 // flashmla.org/de); "原生FP8 调度支持" is item 5 of brainleap's key techniques.
 // The kernels here copy inside one GPU's HBM instead of over NVLink/RDMA.
 //
-// Work unit: one thread owns 16 consecutive hidden values of one token (FP8:
-// two 16-byte loads in, one 16-byte store per copy out) or 8 values (BF16: one
-// 16-byte load, one 16-byte store per copy).  Threads are numbered over the
-// flattened (token, chunk) grid, so a warp reads 512 or 1024 contiguous bytes
-// and every store of a warp covers 512 contiguous bytes of one receive row.
-// For FP8 a 128-value scale block is 8 adjacent lanes; their absmax is
-// combined with three xor-shuffles.  The grid is a multiple of the resident
-// CTAs per SM and loops grid-stride.  Launches use programmatic dependent
-// launch: blocks start while the layout kernels drain and wait (griddepcontrol)
-// before their first global read.
+// FP8, hidden <= 16384 (the bulk kernel).  A CTA owns one token at a time
+// (persistent over tokens), one thread per 16 hidden values: the thread loads
+// its 32 bytes of the row (the next token's 32 bytes are already in flight),
+// the 8 lanes of each 128-value block combine their absmax with xor-shuffles,
+// and the codes go to a shared-memory row (two buffers, alternating).  One
+// thread then hands the row to the TMA engine: k bulk copies, shared ->
+// global, each one whole 7168-byte receive row at hidden 7168, so the copies
+// leave the SM as long contiguous writes without holding registers.  Before a
+// buffer is rewritten, the copies issued from it two tokens earlier must have
+// read it (bulk wait_group.read).  The block leaders store the fp32 scales.
+//
+// BF16, hidden <= 8192 and a multiple of 16: the same staging with BF16 rows.
+// FP8 above 16384 and BF16 otherwise: one thread per 16 or 8 values of the
+// flattened (token, chunk) grid, 16-byte loads and one 16-byte store per copy.  Every
+// kernel launches with programmatic dependent launch: blocks start while the
+// layout drains and wait (griddepcontrol) before their first global read.
 #include "common.cuh"
 #include "launch.h"
 
@@ -24,6 +30,94 @@ namespace cgl {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kMaxBulkHidden = 16384;    // one thread per 16 values: at most 1024 threads
+constexpr int kBulkThreadsPerSM = 1024;  // CTAs per SM of the bulk kernels = this / block size
+constexpr int kMaxBulkHiddenBf16 = 8192; // two staged BF16 rows stay within 32 KiB of shared memory
+
+__device__ __forceinline__ float absmax16(const uint4 a, const uint4 b) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    return m;
+}
+
+// E4M3 codes of the 16 BF16 values in (a, b), each multiplied by inv first.
+__device__ __forceinline__ uint4 quant16(const uint4 a, const uint4 b, float inv) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = cvt_e4m3x2(__fmul_rn(bf16_lo(w[2 * i]), inv), __fmul_rn(bf16_hi(w[2 * i]), inv));
+        const uint32_t hi =
+            cvt_e4m3x2(__fmul_rn(bf16_lo(w[2 * i + 1]), inv), __fmul_rn(bf16_hi(w[2 * i + 1]), inv));
+        q[i] = lo | (hi << 16);
+    }
+    return make_uint4(q[0], q[1], q[2], q[3]);
+}
+
+__global__ void __launch_bounds__(1024)
+dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
+                         const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
+                         float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
+    extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][h] staged code rows
+    griddep_launch_dependents();
+    griddep_wait();                   // dst_pos (and x) may come from the kernels just before
+    const int chunks = h >> 4, nblk = h >> 7;
+    const int c = threadIdx.x;        // this thread's 16 values
+    const bool active = c < chunks;   // only lanes of the last warp can be idle
+    const bool scale_lane = active && (c & 7) == 0;
+    bool bad = false;
+    int buf = 0;
+    int64_t t = blockIdx.x;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (t < n && active) {
+        a = ld_nc_v4(x + t * h + (int64_t)c * 16);
+        b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
+    }
+    for (; t < n; t += gridDim.x, buf ^= 1) {
+        const int64_t tn = t + gridDim.x;   // prefetch the next token's chunk
+        uint4 an = make_uint4(0, 0, 0, 0), bn = an;
+        if (tn < n && active) {
+            an = ld_nc_v4(x + tn * h + (int64_t)c * 16);
+            bn = ld_nc_v4(x + tn * h + (int64_t)c * 16 + 8);
+        }
+        float m = absmax16(a, b);
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        const float amax_c = fmaxf(m, 1e-4f);
+        const float scale = __fdiv_rn(amax_c, 448.0f);
+        const float inv = __fdiv_rn(448.0f, amax_c);
+        const uint4 q = quant16(a, b, inv);
+        uint8_t *row = rows_smem + buf * h;
+        if (threadIdx.x == 0) bulk_wait_read<1>();   // copies from two tokens ago have read `row`
+        __syncthreads();
+        if (active) *reinterpret_cast<uint4 *>(row + c * 16) = q;
+        fence_proxy_async();
+        __syncthreads();
+        const int32_t *dp = dst_pos + t * k;
+        if (threadIdx.x == 0) {
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = __ldg(dp + j);
+                if (r < 0) continue;
+                if (r >= recv_rows) { bad = true; continue; }
+                bulk_store(recv_x + (int64_t)r * h, row, (uint32_t)h);
+            }
+            bulk_commit();
+        }
+        if (scale_lane) {
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = __ldg(dp + j);
+                if (r >= 0 && r < recv_rows) recv_scale[(int64_t)r * nblk + (c >> 3)] = scale;
+            }
+        }
+        a = an;
+        b = bn;
+    }
+    if (threadIdx.x == 0) bulk_wait_all();
+    if (bad) report(status, kErrRange);
+}
 
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
@@ -90,6 +184,59 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
     if (bad) report(status, kErrRange);
 }
 
+// BF16 rows through the same staging: one thread per 16 values, k bulk copies per token.
+__global__ void __launch_bounds__(1024)
+dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
+                          const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
+                          int64_t recv_rows, uint32_t *status) {
+    extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][2h] staged rows
+    griddep_launch_dependents();
+    griddep_wait();
+    const int chunks = h >> 4;
+    const int c = threadIdx.x;
+    const bool active = c < chunks;
+    const uint32_t row_bytes = (uint32_t)h * 2;
+    bool bad = false;
+    int buf = 0;
+    int64_t t = blockIdx.x;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (t < n && active) {
+        a = ld_nc_v4(x + t * h + (int64_t)c * 16);
+        b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
+    }
+    for (; t < n; t += gridDim.x, buf ^= 1) {
+        const int64_t tn = t + gridDim.x;
+        uint4 an = make_uint4(0, 0, 0, 0), bn = an;
+        if (tn < n && active) {
+            an = ld_nc_v4(x + tn * h + (int64_t)c * 16);
+            bn = ld_nc_v4(x + tn * h + (int64_t)c * 16 + 8);
+        }
+        uint8_t *row = rows_smem + (size_t)buf * row_bytes;
+        if (threadIdx.x == 0) bulk_wait_read<1>();
+        __syncthreads();
+        if (active) {
+            reinterpret_cast<uint4 *>(row)[2 * c] = a;
+            reinterpret_cast<uint4 *>(row)[2 * c + 1] = b;
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int32_t *dp = dst_pos + t * k;
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = __ldg(dp + j);
+                if (r < 0) continue;
+                if (r >= recv_rows) { bad = true; continue; }
+                bulk_store(recv_x + (int64_t)r * h, row, row_bytes);
+            }
+            bulk_commit();
+        }
+        a = an;
+        b = bn;
+    }
+    if (threadIdx.x == 0) bulk_wait_all();
+    if (bad) report(status, kErrRange);
+}
+
 __global__ void __launch_bounds__(kThreads)
 dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                      const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
@@ -120,8 +267,22 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
                                int num_sms, uint32_t *status, cudaStream_t stream) {
+    if (n * (h / 16) == 0) return CGL_OK;
+    if (h <= kMaxBulkHidden) {
+        const int threads = (h / 16 + 31) / 32 * 32;
+        const int sms = device_sm_count();
+        if (sms <= 0) return CGL_ECUDA;
+        const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+        int per_sm = kBulkThreadsPerSM / threads;
+        if (per_sm < 1) per_sm = 1;
+        const int64_t want = (int64_t)use_sms * per_sm;
+        const int grid = (int)(n < want ? n : want);
+        const cudaError_t err = launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(threads),
+                                           (size_t)2 * h, stream, x, n, h, k, dst_pos, recv_x,
+                                           recv_scale, recv_rows, status);
+        return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    }
     const int64_t work = n * (h / 16);
-    if (work == 0) return CGL_OK;
     const int grid = copy_grid((const void *)dispatch_fp8_kernel, kThreads,
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;
@@ -133,8 +294,22 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
 cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                 uint16_t *recv_x, int64_t recv_rows, int num_sms, uint32_t *status,
                                 cudaStream_t stream) {
+    if (n * (h / 8) == 0) return CGL_OK;
+    if (h % 16 == 0 && h <= kMaxBulkHiddenBf16) {
+        const int threads = (h / 16 + 31) / 32 * 32;
+        const int sms = device_sm_count();
+        if (sms <= 0) return CGL_ECUDA;
+        const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+        int per_sm = kBulkThreadsPerSM / threads;
+        if (per_sm < 1) per_sm = 1;
+        const int64_t want = (int64_t)use_sms * per_sm;
+        const int grid = (int)(n < want ? n : want);
+        const cudaError_t err = launch_pdl(dispatch_bf16_bulk_kernel, dim3(grid), dim3(threads),
+                                           (size_t)4 * h, stream, x, n, h, k, dst_pos, recv_x,
+                                           recv_rows, status);
+        return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    }
     const int64_t work = n * (h / 8);
-    if (work == 0) return CGL_OK;
     const int grid = copy_grid((const void *)dispatch_bf16_kernel, kThreads,
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;

@@ -44,6 +44,9 @@ size_t layout_workspace_bytes(int64_t n, int E, int R);
 // kernel gets without raising its attribute (host-side bookkeeping on first use).
 bool layout_needs_smem_optin(int E, int R, int k);
 
+// True if the layout for these sizes runs as one cooperative kernel on the current device.
+bool layout_fused_fits(int64_t n, int k, int E, int R);
+
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                          int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
                          int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,

@@ -590,6 +590,12 @@ bool layout_needs_smem_optin(int E, int R, int k) {
     return smem_words(0, k, E, R) * sizeof(int32_t) > kSmemDefault;
 }
 
+bool layout_fused_fits(int64_t n, int k, int E, int R) {
+    const WsLayout w = ws_layout(n, E, R);
+    return smem_words(0, k, E, R) * sizeof(int32_t) <= kSmemDefault && w.blocks <= kMaxFusedBlocks &&
+           w.blocks <= fused_capacity();
+}
+
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                          int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
                          int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
@@ -600,8 +606,8 @@ cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int
     int32_t *ws_r = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.r_off);
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
 
-    const size_t smem0 = smem_words(0, k, E, R) * sizeof(int32_t);
-    if (smem0 <= kSmemDefault && w.blocks <= kMaxFusedBlocks && w.blocks <= fused_capacity()) {
+    if (layout_fused_fits(n, k, E, R)) {
+        const size_t smem0 = smem_words(0, k, E, R) * sizeof(int32_t);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)w.blocks);
         cfg.blockDim = dim3(kThreads);

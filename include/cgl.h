@@ -83,6 +83,14 @@ const char *cgl_status_string(int status);
 size_t cgl_layout_workspace_bytes(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
 
 /*
+ * Number of kernels cgl_get_layout launches for these sizes on the current
+ * device: 1 (one cooperative kernel) when all its blocks fit on the GPU at
+ * once, else 2.  -1 for invalid sizes.  Host-only (queries the device's
+ * occupancy once).
+ */
+int cgl_layout_kernel_count(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
+
+/*
  * cgl_get_layout -- the dispatch layout: how many copies each expert and each
  * logical rank receives, where they start, and the receive row of every
  * (token, slot) copy.  Pages: the dispatch described under "DeepEP是什么" and

@@ -82,7 +82,7 @@ def test_fp8_scales_across_magnitudes(oracle_mod):
 
 def test_fp8_ragged_and_tiny_hidden(oracle_mod):
     rng = np.random.default_rng(5)
-    for n, h, k, E in [(1, 128, 1, 1), (3, 256, 3, 5), (1001, 384, 6, 24), (257, 7168, 8, 256)]:
+    for n, h, k, E in [(1, 128, 1, 1), (3, 256, 3, 5), (1001, 384, 6, 24), (257, 7168, 8, 256), (40, 16512, 2, 8)]:
         x = W.f32_to_bf16_bits(rng.standard_normal((n, h)).astype(np.float32))
         idx = np.stack([rng.permutation(E)[:k] for _ in range(n)]).astype(np.int32)
         idx[rng.random((n, k)) < 0.1] = -1
@@ -107,6 +107,24 @@ def test_dispatch_reports_rows_outside_the_buffer():
     cgl.dispatch_bf16(x, dst, 8, status=st)
     torch.cuda.synchronize()
     assert cgl.status_bits(st) == ["CGL_ERANGE"]
+
+
+def test_bf16_dispatch_shapes(oracle_mod):
+    # staged bulk path (hidden % 16 == 0, <= 8192) and the flattened path (others)
+    rng = np.random.default_rng(8)
+    for n, h, k, E in [(1, 16, 1, 1), (5, 24, 3, 7), (300, 4096, 4, 16), (77, 8200, 2, 4), (33, 9000, 3, 6)]:
+        x = W.f32_to_bf16_bits(rng.standard_normal((n, h)).astype(np.float32))
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(n)]).astype(np.int32)
+        idx[rng.random((n, k)) < 0.1] = -1
+        lay = cgl.get_layout(i32(idx), E, 1)
+        rows = lay.num_recv_rows
+        recv = torch.full((rows, h), 0x1234, dtype=torch.int16, device=dev()).view(torch.bfloat16)
+        cgl.dispatch_bf16(to_bf16(x), lay.dst_pos, rows, recv_x=recv)
+        L = oracle_mod.get_layout(idx, E, 1)
+        ref = oracle_mod.dispatch_bf16(x, L.dst_pos, rows)
+        used = L.recv_src >= 0
+        got = bits(recv)
+        assert np.array_equal(got[used], ref[used]) and np.all(got[~used] == 0x1234)
 
 
 @pytest.mark.parametrize("name", ["tiny", "bf16"])
