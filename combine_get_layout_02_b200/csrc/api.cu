@@ -110,7 +110,7 @@ static bool layout_sizes_ok(int64_t n, int k, int E, int R) {
 
 size_t cgl_layout_workspace_bytes(int64_t n, int k, int E, int R) {
     if (!layout_sizes_ok(n, k, E, R)) return 0;
-    return layout_workspace_bytes(n, E, R);
+    return layout_workspace_bytes(n, k, E, R);
 }
 
 int cgl_layout_kernel_count(int64_t n, int k, int E, int R) {
@@ -131,7 +131,7 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t n, int k, int E, int 
         return CGL_EINVAL;
     if (n > 0 && (!topk_idx || !dst_pos || !is_token_in_rank)) return CGL_EINVAL;
     if (rows > 0 && !recv_src) return CGL_EINVAL;
-    if (workspace_bytes < layout_workspace_bytes(n, E, R)) return CGL_EINVAL;
+    if (workspace_bytes < layout_workspace_bytes(n, k, E, R)) return CGL_EINVAL;
     if (!aligned(topk_idx, 4) || !aligned(tokens_per_expert, 4) || !aligned(tokens_per_rank, 4) ||
         !aligned(expert_offset, 4) || !aligned(max_count, 4) || !aligned(dst_pos, 4) ||
         !aligned(recv_src, 4) || !aligned(status_dev, 4) || !aligned(is_token_in_rank, 16) ||

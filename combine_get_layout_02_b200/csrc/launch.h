@@ -38,7 +38,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-size_t layout_workspace_bytes(int64_t n, int E, int R);
+size_t layout_workspace_bytes(int64_t n, int k, int E, int R);
 
 // True if some layout kernel for these sizes needs more shared memory than a
 // kernel gets without raising its attribute (host-side bookkeeping on first use).

@@ -130,7 +130,7 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
                           size_t workspace_bytes, uint32_t *status_dev, void *stream);
 
 /* Size of the device scratch array behind cgl_get_layout_noalloc. */
-#define CGL_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+#define CGL_NOALLOC_SCRATCH_BYTES (512u * 1024u)
 
 /*
  * cgl_get_layout_noalloc -- cgl_get_layout for callers that cannot allocate
@@ -145,17 +145,17 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
  *
  * Same arguments, outputs, ordering and errors as cgl_get_layout, minus the
  * workspace: the scratch is a fixed device array of CGL_NOALLOC_SCRATCH_BYTES
- * (256 KiB) inside libcgl.so, held by every GPU that loads the library until
+ * (512 KiB) inside libcgl.so, held by every GPU that loads the library until
  * the process exits.  The call allocates nothing (no cudaMalloc or cudaFree,
  * no allocating library routine); the caller still passes every input and
  * output buffer.
  * Limits, rejected with CGL_EINVAL before anything is launched:
  *   cgl_layout_workspace_bytes(...) <= CGL_NOALLOC_SCRATCH_BYTES
- *     (at E = 256, R = 64: up to 51,968 tokens), and
- *   256 * (num_topk | 1) + 12 * num_experts + num_ranks
- *     + (num_ranks > 64 ? 256 * ceil(num_ranks / 32) : 0) <= 12032
- *     (the layout kernels then fit in the default 48 KiB of shared memory per
- *     block; with num_ranks <= 64: any num_topk up to E = 293, num_topk <= 8 up to E = 805).
+ *     (at E = 256, R = 64, num_topk = 8: up to 52,096 tokens), and
+ *   12 * num_experts + num_ranks + T * ceil(num_ranks / 32) <= 9984, with
+ *     T = min(256, 1024 / num_topk) tokens per block (the layout kernels then
+ *     fit in the default 48 KiB of shared memory per block; with
+ *     num_ranks <= 64 this holds for any num_topk up to E = 784).
  * Set-up: the first call on a device (with that device current) looks up the
  * array's device address once and caches it; make that first call before any
  * stream capture.  CGL_ECUDA if the lookup fails.
