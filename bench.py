@@ -269,6 +269,25 @@ class GpuStep:
         return e
 
 
+def capture_step(step: GpuStep):
+    """One step's launches captured into a CUDA graph (on a side stream, after two eager runs)."""
+    import torch
+
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            step.run()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step.run()
+    torch.cuda.synchronize()
+    return g
+
+
 def run_e2e(step: GpuStep, steps: int):
     """Same step through the public API with host buffers: pinned H2D of the
     step's inputs, the kernels, D2H of the combined output and the counts."""
@@ -419,8 +438,12 @@ def run_ours(args):
     step = GpuStep(wl, rank_seed(args.seed, rank), dev)
     phases = step.kernels()
 
+    graph = None if args.no_graph else capture_step(step)
     for _ in range(args.warmup):
-        step.run()
+        if graph is not None:
+            graph.replay()
+        else:
+            step.run()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -429,12 +452,17 @@ def run_ours(args):
         sampler.start()
         time.sleep(0.3)   # let nvidia-smi start sampling before the timed region
     # timed region: K steps, one event on each side, nothing between the kernels
-    # (an event between two kernels stops the next one from launching early)
+    # (an event between two kernels stops the next one from launching early);
+    # by default each step is one replay of a CUDA graph holding the step's launches
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record()
-    for _ in range(args.steps):
-        step.run()
+    if graph is not None:
+        for _ in range(args.steps):
+            graph.replay()
+    else:
+        for _ in range(args.steps):
+            step.run()
     e_end.record()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
@@ -490,6 +518,7 @@ def run_ours(args):
         "value": value, "ms_per_step": ms, "roofline": roof, "kernels": kernels,
         "dispatch_plus_combine_us": sum(kernels[n]["us"] for n in kernels if n != "layout"),
         "gpu_launches": args.steps * sum(p[1] for p in phases),
+        "launch": "eager" if args.no_graph else "CUDA graph of one step, replayed K times (e2e and per-kernel passes eager)",
         "kernel_timing": ("per-kernel us from a second pass of the same K steps with a CUDA event "
                           f"after every kernel ({ms_instr * 1e3:.1f} us/step there vs {ms * 1e3:.1f} clean); "
                           "each includes the launch gap the events add"),
@@ -524,6 +553,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -34,14 +34,15 @@
 //
 // Launch shapes.  With one block (up to 1024 pairs, e.g. 128 decode tokens at
 // k = 8) the block's own counts are the totals and nothing is exchanged.
-// When every block fits on the GPU at once, one cooperative kernel does everything and the blocks exchange their counts through the
-// workspace: each block writes its row, then release-stores a 64-bit tag
-// unique to the call into its flag word, and waits, with a bounded spin
-// (CGL_ETIMEOUT after ~1 s), until every flag shows that tag.  Otherwise two
-// kernels run (counts, then bases + rows), the second with programmatic
-// dependent launch; it recomputes the cheap in-warp ranks.
-#include <atomic>
-#include <chrono>
+// When every block fits on the GPU at once, one cooperative kernel does
+// everything and the blocks exchange their counts through the workspace: each
+// block writes its row, then release-stores this launch's 64-bit tag into its
+// flag word, and waits, with a bounded spin (CGL_ETIMEOUT after ~1 s), until
+// every flag shows that tag.  The tag is a generation counter kept in the
+// workspace (+1 per launch), so it changes on every launch, replays of a
+// captured graph included.  Otherwise two kernels run (counts, then bases +
+// rows), the second with programmatic dependent launch; it recomputes the
+// cheap in-warp ranks.
 #include <mutex>
 
 #include "common.cuh"
@@ -68,7 +69,8 @@ __host__ __device__ __forceinline__ int tokens_per_block(int k) {
 }
 __host__ __device__ __forceinline__ int mask_words(int R) { return (R + 31) >> 5; }
 
-// Workspace: [flags: blocks x u64][pad to 256 B][expert counts: blocks x E][pad][rank counts: blocks x R]
+// Workspace: [generation: u64][flags: blocks x u64][pad to 256 B][expert counts: blocks x E][pad]
+//            [rank counts: blocks x R]
 struct WsLayout {
     int64_t blocks;
     size_t e_off, r_off, bytes;
@@ -80,7 +82,7 @@ WsLayout ws_layout(int64_t n, int k, int E, int R) {
     WsLayout w;
     const int T = tokens_per_block(k);
     w.blocks = n > 0 ? (n + T - 1) / T : 1;
-    w.e_off = align256((size_t)w.blocks * sizeof(uint64_t));
+    w.e_off = align256((size_t)(w.blocks + 1) * sizeof(uint64_t));
     w.r_off = w.e_off + align256((size_t)w.blocks * (size_t)E * sizeof(int32_t));
     w.bytes = w.r_off + (size_t)w.blocks * (size_t)R * sizeof(int32_t);
     return w;
@@ -89,6 +91,17 @@ WsLayout ws_layout(int64_t n, int k, int E, int R) {
 __device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Flags hold this constant in their high half; counts (non-negative int32) never do.
+constexpr uint64_t kTagHigh = 0x9E3779B9ull << 32;
+
 __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
     uint64_t v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -476,7 +489,7 @@ __device__ void zero_words(int32_t *p, int n) {
 
 __global__ void __launch_bounds__(kThreads)
 layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap,
-                    uint64_t *flags, int32_t *ws_e, int32_t *ws_r, uint64_t tag,
+                    uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
                     int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                     uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
                     int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
@@ -488,6 +501,13 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const int nb = gridDim.x, b = blockIdx.x;
 
     griddep_launch_dependents();   // the copy kernels may get resident; they wait for this grid
+    // This launch's tag: generation + 1.  Every block reads the generation before
+    // it publishes its flag, and block 0 advances it only after it has seen every
+    // flag, so all blocks agree and the next launch (a graph replay too) gets a new tag.
+    uint64_t *gen = flags;
+    flags += 1;
+    const uint64_t g0 = ld_relaxed_u64(gen) & 0xFFFFFFFFull;
+    const uint64_t tag = kTagHigh | ((g0 + 1) & 0xFFFFFFFFull);
     zero_words(s.wc, kWarps * E);
     zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
     zero_words(s.hr, R);
@@ -529,6 +549,7 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         if (tid == 0) report(status, 1u << CGL_ETIMEOUT);
         return;
     }
+    if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
     bases_and_rows<true>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert, tokens_per_rank,
                          expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp);
 }
@@ -604,21 +625,6 @@ int fused_capacity() {
     return per_sm > 0 ? per_sm * device_sm_count() : 0;
 }
 
-// A 64-bit tag unique to each call: a per-process salt (never 0) in the high
-// half and a call counter in the low half, so no flag left by another call,
-// and no freshly zeroed memory, can match it.
-uint64_t next_tag() {
-    static std::atomic<uint64_t> counter{0};
-    static const uint64_t salt = [] {
-        uint64_t v = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
-        v ^= v >> 29;
-        v *= 0xBF58476D1CE4E5B9ull;
-        v ^= v >> 32;
-        return (v & 0xFFFFFFFFull) | 1ull;
-    }();
-    return (salt << 32) | ((counter.fetch_add(1) + 1) & 0xFFFFFFFFull);
-}
-
 }  // namespace
 
 size_t layout_workspace_bytes(int64_t n, int k, int E, int R) { return ws_layout(n, k, E, R).bytes; }
@@ -654,7 +660,7 @@ cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const cudaError_t err = cudaLaunchKernelEx(
-            &cfg, layout_fused_kernel, idx, n, k, E, R, cap, flags, ws_e, ws_r, next_tag(),
+            &cfg, layout_fused_kernel, idx, n, k, E, R, cap, flags, ws_e, ws_r,
             tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src,
             recv_rows, status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;

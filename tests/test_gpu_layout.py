@@ -120,3 +120,34 @@ def test_layout_two_kernel_path_large_shared_memory_with_duplicates(oracle_mod):
     idx[:, 5] = idx[:, 3]                      # every token repeats one expert
     run_both(oracle_mod, idx, E, R, 0)
     run_both(oracle_mod, idx, E, R, 64)
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_layout_graph_replays_with_changing_ids(oracle_mod, name):
+    # one captured launch, replayed with different ids: every replay must see its
+    # own blocks' counts (the inter-block exchange is tagged per launch on the device)
+    wl = W.WORKLOADS[name]
+    E, R = wl.num_experts, wl.num_ranks
+    ids = [W.make_inputs(name, seed).topk_idx for seed in (1, 2, 3)]
+    idx = i32(ids[0])
+    ws = torch.empty(cgl.layout_workspace_bytes(wl.num_tokens, wl.topk, E, R), dtype=torch.uint8, device=dev())
+    lay = cgl.get_layout(idx, E, R, workspace=ws)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        cgl.get_layout(idx, E, R, workspace=ws, out=lay)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cgl.get_layout(idx, E, R, workspace=ws, out=lay)
+    for a in (ids[1], ids[2], ids[0], ids[1]):
+        idx.copy_(torch.from_numpy(a))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle_mod.get_layout(a, E, R)
+        assert np.array_equal(lay.dst_pos.cpu().numpy(), ref.dst_pos)
+        assert np.array_equal(lay.expert_offset.cpu().numpy(), ref.expert_offset)
+        assert np.array_equal(lay.recv_src.cpu().numpy(), ref.recv_src)
+        assert np.array_equal(lay.tokens_per_rank.cpu().numpy(), ref.tokens_per_rank)
+    del g
