@@ -172,19 +172,21 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- steps
 
-def workload_label(wl: W.Workload) -> str:
-    return f"{wl.name}: {wl.description}"
+def workload_label(wl: W.Workload, dedup: bool = False) -> str:
+    tail = "; per-rank deduplicated dispatch (one copy per token and rank)" if dedup else ""
+    return f"{wl.name}: {wl.description}{tail}"
 
 
 class GpuStep:
     """Device buffers for one workload and the launch sequence of one step."""
 
-    def __init__(self, wl: W.Workload, seed: int, device):
+    def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False):
         import torch
 
         import combine_get_layout_02_b200 as cgl
 
         self.cgl, self.torch, self.wl, self.dev = cgl, torch, wl, device
+        self.dedup = dedup
         inp = W.make_inputs(wl, seed)
         n, h, k = wl.num_tokens, wl.hidden, wl.topk
         self.host = inp
@@ -220,14 +222,39 @@ class GpuStep:
             self.recv_x = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
             self.grad_recv = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((n, h), dtype=torch.bfloat16, device=device)
-        torch.cuda.synchronize(device)
         self.bytes = W.algorithmic_bytes(wl)
+        if dedup:
+            # one copy per (token, destination rank); the combine sums each rank's partial row
+            rcap = 0
+            if wl.padded:
+                rcap = int(cgl.get_rank_layout(self.idx, E, R, 0, workspace=self.ws).max_count.item())
+            self.rcap = rcap
+            self.rlay = cgl.get_rank_layout(self.idx, E, R, rcap, workspace=self.ws, status=self.status)
+            self.rrows = self.rlay.num_recv_rows
+            self.w_rank = (self.rlay.rank_dst >= 0).float()
+            used = int(self.rlay.rank_offset[-1].item())
+            self.used_rank_rows = used
+            nb = wl.num_tokens
+            self.bytes = {
+                "layout": 12 * nb * k,
+                "dispatch_fp8": 2 * nb * h + 4 * nb * k + used * (h + 4 * (h // 128)),
+                "dispatch_bf16": 2 * nb * h + 4 * nb * k + used * 2 * h,
+                "combine": 2 * used * h + 8 * nb * k + 2 * nb * h,
+            }
+            if wl.padded:
+                self.y = self.y.new_zeros((self.rrows, h))
+                self.y[self.rlay.rank_dst[self.rlay.rank_dst >= 0].long()] = \
+                    bf16(y_host[:used]).to(device)
+        torch.cuda.synchronize(device)
 
     def kernels(self):
         """(name, launches per step, algorithmic bytes per launch) of each step phase."""
         b = self.bytes
         wl = self.wl
-        nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_experts, wl.num_ranks)
+        if self.dedup:   # rank keys: the layout of an E = R problem
+            nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_ranks, wl.num_ranks)
+        else:
+            nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_experts, wl.num_ranks)
         ph = [("layout", nl, b["layout"])]
         if self.wl.fp8:
             ph.append(("dispatch_fp8", 1, b["dispatch_fp8"]))
@@ -247,6 +274,23 @@ class GpuStep:
         E, R = wl.num_experts, wl.num_ranks
         rec = (lambda: events.append(self._event())) if events is not None else (lambda: None)
         rec()
+        if self.dedup:
+            cgl.get_rank_layout(self.idx, E, R, self.rcap, workspace=self.ws, out=self.rlay, status=self.status)
+            rec()
+            if wl.fp8:
+                cgl.dispatch_fp8(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
+                                 recv_scale=self.recv_scale, status=self.status)
+            else:
+                cgl.dispatch_bf16(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
+                                  status=self.status)
+            rec()
+            cgl.combine(self.y, self.rlay.rank_dst, self.w_rank, out=self.out, status=self.status)
+            rec()
+            if wl.with_grad:
+                cgl.dispatch_bf16(self.grad, self.rlay.rank_dst, self.rrows, recv_x=self.grad_recv,
+                                  status=self.status)
+                rec()
+            return
         cgl.get_layout(self.idx, E, R, self.cap, workspace=self.ws, out=self.lay, status=self.status)
         rec()
         if wl.fp8:
@@ -377,7 +421,7 @@ def base_line(args, wl, n_gpus):
         "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": {
-            "workload": workload_label(wl), "num_tokens": wl.num_tokens, "hidden": wl.hidden,
+            "workload": workload_label(wl, getattr(args, "dedup", False)), "num_tokens": wl.num_tokens, "hidden": wl.hidden,
             "num_experts": wl.num_experts, "num_groups": wl.num_groups, "topk_group": wl.topk_group,
             "topk": wl.topk, "num_ranks": wl.num_ranks,
             "storage": ("x bf16 -> e4m3 rows + f32 1x128 scales; combine bf16 in, f32 accumulate, bf16 out"
@@ -435,7 +479,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     dist_init("nccl")
     wl = W.WORKLOADS[args.workload]
-    step = GpuStep(wl, rank_seed(args.seed, rank), dev)
+    step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup)
     phases = step.kernels()
 
     graph = None if args.no_graph else capture_step(step)
@@ -526,7 +570,7 @@ def run_ours(args):
     })
     if e2e:
         line["e2e"] = e2e
-    if not args.no_cpu_baseline and world == 1:
+    if not args.no_cpu_baseline and world == 1 and not args.dedup:
         import oracle
 
         threads = oracle.set_threads(cpu_threads())
@@ -553,6 +597,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--dedup", action="store_true",
+                    help="per-rank deduplicated dispatch: one copy per (token, rank), rank-sum combine")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -26,7 +26,7 @@ from typing import NamedTuple, Optional
 import torch
 
 __all__ = [
-    "CglError", "Layout", "lib", "get_layout", "dispatch_fp8", "dispatch_bf16", "combine",
+    "CglError", "Layout", "RankLayout", "lib", "get_layout", "get_rank_layout", "dispatch_fp8", "dispatch_bf16", "combine",
     "layout_workspace_bytes", "layout_kernel_count", "status_bits", "check_status", "new_status",
 ]
 
@@ -74,6 +74,8 @@ def lib():
         L.cgl_layout_kernel_count.restype = I
         L.cgl_get_layout.argtypes = [P, I64, I, I, I, OP, P, P, P, P, P, P, P, P, C.c_size_t, P, P]
         L.cgl_get_layout.restype = I
+        L.cgl_get_rank_layout.argtypes = [P, I64, I, I, I, OP, P, P, P, P, P, P, C.c_size_t, P, P]
+        L.cgl_get_rank_layout.restype = I
         L.cgl_dispatch_fp8.argtypes = [P, I64, I, I, P, P, P, I64, OP, P, P]
         L.cgl_dispatch_fp8.restype = I
         L.cgl_dispatch_bf16.argtypes = [P, I64, I, I, P, P, I64, OP, P, P]
@@ -191,6 +193,46 @@ def get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, capacit
         _ptr(out.max_count), _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
     _check(code, "cgl_get_layout")
+    return out
+
+
+class RankLayout(NamedTuple):
+    tokens_per_rank: torch.Tensor     # int32 [R]
+    rank_offset: torch.Tensor         # int32 [R + 1]
+    max_count: torch.Tensor           # int32 [1]
+    rank_dst: torch.Tensor            # int32 [N, k]  (row per first slot on each rank, else -1)
+    recv_token: torch.Tensor          # int32 [num_recv_rows]
+    num_recv_rows: int                # N*k (compact) or R*capacity (padded)
+    capacity: int
+
+
+def get_rank_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, capacity: int = 0, *,
+                    status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    out: Optional[RankLayout] = None, stream=None) -> RankLayout:
+    """One copy per (token, destination rank): the deduplicated layout (cgl_get_rank_layout)."""
+    idx = _dev(topk_idx, "topk_idx", torch.int32, 2)
+    n, k = idx.shape
+    E, R = int(num_experts), int(num_ranks)
+    dev = idx.device
+    rows = R * capacity if capacity > 0 else n * k
+    ws_bytes = layout_workspace_bytes(n, k, R, R)
+    if ws_bytes == 0 or E % R:
+        raise CglError(EINVAL, "get_rank_layout", "invalid sizes")
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = RankLayout(
+            torch.empty(R, dtype=torch.int32, device=dev),
+            torch.empty(R + 1, dtype=torch.int32, device=dev),
+            torch.empty(1, dtype=torch.int32, device=dev),
+            torch.empty((n, k), dtype=torch.int32, device=dev),
+            torch.empty(rows, dtype=torch.int32, device=dev),
+            rows, int(capacity))
+    code = lib().cgl_get_rank_layout(
+        _ptr(idx), n, k, E, R, _opts(0, capacity), _ptr(out.tokens_per_rank), _ptr(out.rank_offset),
+        _ptr(out.max_count), _ptr(out.rank_dst), _ptr(out.recv_token), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(code, "cgl_get_rank_layout")
     return out
 
 

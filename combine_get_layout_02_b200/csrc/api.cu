@@ -142,6 +142,28 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t n, int k, int E, int 
                          status_dev, static_cast<cudaStream_t>(stream));
 }
 
+cgl_status cgl_get_rank_layout(const int32_t *topk_idx, int64_t n, int k, int E, int R,
+                               const cgl_opts *opts, int32_t *tokens_per_rank, int32_t *rank_offset,
+                               int32_t *max_count, int32_t *rank_dst, int32_t *recv_token,
+                               void *workspace, size_t workspace_bytes, uint32_t *status_dev,
+                               void *stream) {
+    if (!layout_sizes_ok(n, k, E, R)) return CGL_EINVAL;
+    const int cap = opt_cap(opts);
+    if (cap < 0 || (int64_t)R * cap >= ((int64_t)1 << 31)) return CGL_EINVAL;
+    const int64_t rows = cap > 0 ? (int64_t)R * cap : n * k;
+    if (!tokens_per_rank || !rank_offset || !max_count || !workspace) return CGL_EINVAL;
+    if (n > 0 && (!topk_idx || !rank_dst)) return CGL_EINVAL;
+    if (rows > 0 && !recv_token) return CGL_EINVAL;
+    if (workspace_bytes < layout_workspace_bytes(n, k, R, R)) return CGL_EINVAL;
+    if (!aligned(topk_idx, 4) || !aligned(tokens_per_rank, 4) || !aligned(rank_offset, 4) ||
+        !aligned(max_count, 4) || !aligned(rank_dst, 4) || !aligned(recv_token, 4) ||
+        !aligned(status_dev, 4) || !aligned(workspace, 16))
+        return CGL_EALIGN;
+    return launch_rank_layout(topk_idx, n, k, E, R, cap, tokens_per_rank, rank_offset, max_count,
+                              rank_dst, recv_token, workspace, status_dev,
+                              static_cast<cudaStream_t>(stream));
+}
+
 cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                             uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
                             const cgl_opts *opts, uint32_t *status_dev, void *stream) {

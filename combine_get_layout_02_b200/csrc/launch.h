@@ -52,6 +52,12 @@ cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int
                          int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
                          int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream);
 
+// Per-rank layout: keys are destination ranks (one row per token and rank).
+cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                              int32_t *tokens_per_rank, int32_t *rank_offset, int32_t *max_count,
+                              int32_t *rank_dst, int32_t *recv_token, void *ws, uint32_t *status,
+                              cudaStream_t stream);
+
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
                                int num_sms, uint32_t *status, cudaStream_t stream);

@@ -156,10 +156,14 @@ struct Pairs {
 __device__ __forceinline__ int pair_of(int i) { return (threadIdx.x >> 5) * (kChunks * 32) + i * 32 + (threadIdx.x & 31); }
 
 // Load this thread's ids (coalesced: each warp reads 32 consecutive ids per
-// chunk) and rank them within the warp.  s.wc must be zero.  Returns true if
-// an id outside [-1, E) was seen (such slots make no copy).
-__device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k, int E, const Smem &s,
-                              Pairs &P) {
+// chunk), turn them into keys and rank the keys within the warp.  Expert mode:
+// key = expert id.  Rank mode (kRankKeys): key = the expert's rank e / key_div
+// for the first slot of the token on that rank, else -1 (one copy per token
+// and rank).  Keys index s.wc[.][0, nkeys).  s.wc must be zero.  Returns true
+// if an id outside [-1, E_ids) was seen (such slots make no copy).
+template <bool kRankKeys>
+__device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids, int key_div,
+                              int nkeys, const Smem &s, Pairs &P) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int T = tokens_per_block(k);
     P.t0 = (int64_t)blockIdx.x * T;
@@ -175,9 +179,25 @@ __device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k,
     }
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
-        if (P.e[i] < -1 || P.e[i] >= E) { bad = true; P.e[i] = -1; }
+        if (P.e[i] < -1 || P.e[i] >= E_ids) { bad = true; P.e[i] = -1; }
     }
-    int32_t *wc = s.wc + warp * E;
+    if (kRankKeys) {
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) {
+            const int32_t e = P.e[i];
+            if (e < 0) continue;
+            const int p = pair_of(i);
+            const int tl = p / k, j = p - tl * k;
+            const int r = e / key_div;
+            bool first = true;
+            for (int jj = 0; jj < j; ++jj) {
+                const int32_t e2 = __ldg(src + tl * k + jj);
+                if (e2 >= 0 && e2 < E_ids && e2 / key_div == r) first = false;
+            }
+            P.e[i] = first ? r : -1;
+        }
+    }
+    int32_t *wc = s.wc + warp * nkeys;
     const uint32_t lower = (1u << lane) - 1u;
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
@@ -401,7 +421,7 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
 }
 
 // Bases, the global outputs (block 0) and the rows of the block's pairs.
-template <bool kCoherent>
+template <bool kCoherent, bool kRankKeys>
 __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t n, int k, int E, int R,
                                int cap, int64_t recv_rows, int32_t *__restrict__ tokens_per_expert,
                                int32_t *__restrict__ tokens_per_rank, int32_t *__restrict__ expert_offset,
@@ -440,7 +460,8 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
             *max_count = m;
         }
         // tokens_per_rank: column sums of the rank table (s.part is free again)
-        if (nb == 1 && s.hr != nullptr) {
+        if (tokens_per_rank == nullptr) {
+        } else if (nb == 1 && s.hr != nullptr) {
             for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
         } else {
             column_sums<kCoherent>(ws_r, nb, R, 0, s.off, nullptr, s.part);
@@ -475,7 +496,8 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         }
         const int64_t q = P.t0 * k + p;
         dst_pos[q] = d;
-        if (d >= 0) recv_src[d] = (int32_t)q;
+        // expert mode: the row's source slot t*k + j; rank mode: its source token t
+        if (d >= 0) recv_src[d] = kRankKeys ? (int32_t)(P.t0 + p / k) : (int32_t)q;
     }
     if (over) report(status, kErrCapacity);
     if (bad_row) report(status, kErrRange);
@@ -487,9 +509,13 @@ __device__ void zero_words(int32_t *p, int n) {
 
 // ------------------------------------------------------------------ kernels
 
+// Kernel arguments: E = number of keys (experts, or ranks in rank mode),
+// E_ids / key_div = valid id range and expert-to-rank divisor for the key
+// transform.  in_rank == nullptr skips the rank sets (rank mode).
+template <bool kRankKeys>
 __global__ void __launch_bounds__(kThreads)
-layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap,
-                    uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
+                    int key_div, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
                     int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                     uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
                     int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
@@ -499,6 +525,7 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const Smem s = carve(0, smem_fused, k, E, R);
     const int tid = threadIdx.x;
     const int nb = gridDim.x, b = blockIdx.x;
+    const bool with_ranks = in_rank != nullptr;
 
     griddep_launch_dependents();   // the copy kernels may get resident; they wait for this grid
     // This launch's tag: generation + 1.  Every block reads the generation before
@@ -513,17 +540,20 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     zero_words(s.hr, R);
     __syncthreads();
     Pairs P;
-    const bool bad = load_and_rank(idx, n, k, E, s, P);
-    rank_sets(k, E, R, s, P);
+    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
+    if (with_ranks) rank_sets(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
-    rank_counts(k, R, s, P);
-    write_rank_rows(R, in_rank, s, P);
+    if (with_ranks) {
+        rank_counts(k, R, s, P);
+        write_rank_rows(R, in_rank, s, P);
+    }
     __syncthreads();
     if (nb == 1) {   // nothing to exchange
         if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
-        bases_and_rows<true>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert, tokens_per_rank,
-                             expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp);
+        bases_and_rows<true, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+                                        tokens_per_rank, expert_offset, max_count, dst_pos, recv_src,
+                                        status, s, P, scan_tmp);
         return;
     }
     for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
@@ -550,38 +580,44 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         return;
     }
     if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
-    bases_and_rows<true>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert, tokens_per_rank,
-                         expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp);
+    bases_and_rows<true, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+                                    tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
+                                    s, P, scan_tmp);
 }
 
+template <bool kRankKeys>
 __global__ void __launch_bounds__(kThreads)
-layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R,
+layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int E_ids, int key_div,
                     int32_t *__restrict__ ws_e, int32_t *__restrict__ ws_r,
                     uint8_t *__restrict__ in_rank, uint32_t *status) {
     extern __shared__ __align__(16) int32_t smem_count[];
     const Smem s = carve(1, smem_count, k, E, R);
     const int tid = threadIdx.x;
+    const bool with_ranks = in_rank != nullptr;
     griddep_launch_dependents();   // the rows kernel may start; it waits for this grid
     zero_words(s.wc, kWarps * E);
     zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
     zero_words(s.hr, R);
     __syncthreads();
     Pairs P;
-    const bool bad = load_and_rank(idx, n, k, E, s, P);
-    rank_sets(k, E, R, s, P);
+    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
+    if (with_ranks) rank_sets(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
-    rank_counts(k, R, s, P);
-    write_rank_rows(R, in_rank, s, P);
+    if (with_ranks) {
+        rank_counts(k, R, s, P);
+        write_rank_rows(R, in_rank, s, P);
+    }
     __syncthreads();
     for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)blockIdx.x * E + i] = s.he[i];
     for (int i = tid; i < R; i += kThreads) ws_r[(int64_t)blockIdx.x * R + i] = s.hr[i];
     if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
 }
 
+template <bool kRankKeys>
 __global__ void __launch_bounds__(kThreads)
-layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap,
-                   const int32_t *__restrict__ ws_e, const int32_t *__restrict__ ws_r,
+layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
+                   int key_div, const int32_t *__restrict__ ws_e, const int32_t *__restrict__ ws_r,
                    int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                    int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
                    int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
@@ -595,34 +631,43 @@ layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int
     // topk_idx is not written by the counts kernel, which started only after
     // everything before it in the stream had finished: it may be read before the wait
     Pairs P;
-    load_and_rank(idx, n, k, E, s, P);
+    load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
     __syncthreads();
     warp_offsets(E, s);
     griddep_wait();
     __syncthreads();
-    bases_and_rows<false>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert, tokens_per_rank,
-                          expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp);
+    bases_and_rows<false, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+                                     tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
+                                     s, P, scan_tmp);
 }
 
 // ------------------------------------------------------------------ host side
 
 std::mutex g_mu;
-int g_fused_ctas_per_sm[64] = {0};   // fused-kernel occupancy at kSmemDefault, per device (-1: none)
+int g_fused_ctas_per_sm[2][64] = {{0}};   // fused-kernel occupancy at kSmemDefault, per mode and device
 
 // Largest grid of the fused kernel that is certain to be co-resident; 0 if none.
+template <bool kRankKeys>
 int fused_capacity() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_fused_ctas_per_sm[dev] == 0) {
+    int &slot = g_fused_ctas_per_sm[kRankKeys ? 1 : 0][dev];
+    if (slot == 0) {
         int v = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, layout_fused_kernel, kThreads,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, layout_fused_kernel<kRankKeys>, kThreads,
                                                           kSmemDefault) != cudaSuccess)
             return 0;
-        g_fused_ctas_per_sm[dev] = v > 0 ? v : -1;
+        slot = v > 0 ? v : -1;
     }
-    const int per_sm = g_fused_ctas_per_sm[dev];
-    return per_sm > 0 ? per_sm * device_sm_count() : 0;
+    return slot > 0 ? slot * device_sm_count() : 0;
+}
+
+template <bool kRankKeys>
+bool fused_fits(int64_t n, int k, int nkeys, int R) {
+    const WsLayout w = ws_layout(n, k, nkeys, R);
+    return smem_words(0, k, nkeys, R) * sizeof(int32_t) <= kSmemDefault &&
+           w.blocks <= fused_capacity<kRankKeys>();
 }
 
 }  // namespace
@@ -633,22 +678,22 @@ bool layout_needs_smem_optin(int E, int R, int k) {
     return smem_words(0, k, E, R) * sizeof(int32_t) > kSmemDefault;
 }
 
-bool layout_fused_fits(int64_t n, int k, int E, int R) {
-    const WsLayout w = ws_layout(n, k, E, R);
-    return !layout_needs_smem_optin(E, R, k) && w.blocks <= fused_capacity();
-}
+bool layout_fused_fits(int64_t n, int k, int E, int R) { return fused_fits<false>(n, k, E, R); }
 
-cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
-                         int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
-                         int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
-                         int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+template <bool kRankKeys>
+cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
+                              int32_t *tokens_per_key, int32_t *tokens_per_rank, uint8_t *in_rank,
+                              int32_t *key_offset, int32_t *max_count, int32_t *dst_pos,
+                              int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+    const int E = kRankKeys ? R : E_ids;        // number of keys
+    const int key_div = E_ids / R;
     const WsLayout w = ws_layout(n, k, E, R);
     uint64_t *flags = static_cast<uint64_t *>(ws);
     int32_t *ws_e = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.e_off);
     int32_t *ws_r = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.r_off);
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
 
-    if (layout_fused_fits(n, k, E, R)) {
+    if (fused_fits<kRankKeys>(n, k, E, R)) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)w.blocks);
         cfg.blockDim = dim3(kThreads);
@@ -660,24 +705,43 @@ cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const cudaError_t err = cudaLaunchKernelEx(
-            &cfg, layout_fused_kernel, idx, n, k, E, R, cap, flags, ws_e, ws_r,
-            tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src,
-            recv_rows, status);
+            &cfg, layout_fused_kernel<kRankKeys>, idx, n, k, E, R, cap, E_ids, key_div, flags, ws_e, ws_r,
+            tokens_per_key, tokens_per_rank, in_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
+            status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
     }
 
     const size_t smem1 = smem_words(1, k, E, R) * sizeof(int32_t);
     const size_t smem2 = smem_words(2, k, E, R) * sizeof(int32_t);
-    if (smem1 > kSmemDefault && !ensure_smem_attr((const void *)layout_count_kernel, smem1)) return CGL_ECUDA;
-    if (smem2 > kSmemDefault && !ensure_smem_attr((const void *)layout_rows_kernel, smem2)) return CGL_ECUDA;
-    layout_count_kernel<<<(unsigned)w.blocks, kThreads, smem1, stream>>>(idx, n, k, E, R, ws_e, ws_r,
-                                                                          in_rank, status);
+    if (smem1 > kSmemDefault && !ensure_smem_attr((const void *)layout_count_kernel<kRankKeys>, smem1))
+        return CGL_ECUDA;
+    if (smem2 > kSmemDefault && !ensure_smem_attr((const void *)layout_rows_kernel<kRankKeys>, smem2))
+        return CGL_ECUDA;
+    layout_count_kernel<kRankKeys><<<(unsigned)w.blocks, kThreads, smem1, stream>>>(
+        idx, n, k, E, R, E_ids, key_div, ws_e, ws_r, in_rank, status);
     if (cudaGetLastError() != cudaSuccess) return CGL_ECUDA;
-    const cudaError_t err = launch_pdl(layout_rows_kernel, dim3((unsigned)w.blocks), dim3(kThreads), smem2,
-                                       stream, idx, n, k, E, R, cap, (const int32_t *)ws_e,
-                                       (const int32_t *)ws_r, tokens_per_expert, tokens_per_rank,
-                                       expert_offset, max_count, dst_pos, recv_src, recv_rows, status);
+    const cudaError_t err = launch_pdl(layout_rows_kernel<kRankKeys>, dim3((unsigned)w.blocks), dim3(kThreads),
+                                       smem2, stream, idx, n, k, E, R, cap, E_ids, key_div,
+                                       (const int32_t *)ws_e, (const int32_t *)ws_r, tokens_per_key,
+                                       tokens_per_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
+                                       status);
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+}
+
+cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                         int32_t *tokens_per_expert, int32_t *tokens_per_rank, uint8_t *in_rank,
+                         int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
+                         int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+    return launch_layout_impl<false>(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
+                                     expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
+}
+
+cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                              int32_t *tokens_per_rank, int32_t *rank_offset, int32_t *max_count,
+                              int32_t *rank_dst, int32_t *recv_token, void *ws, uint32_t *status,
+                              cudaStream_t stream) {
+    return launch_layout_impl<true>(idx, n, k, E, R, cap, tokens_per_rank, nullptr, nullptr, rank_offset,
+                                    max_count, rank_dst, recv_token, ws, status, stream);
 }
 
 }  // namespace cgl

@@ -129,6 +129,41 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
                           int32_t *dst_pos, int32_t *recv_src, void *workspace,
                           size_t workspace_bytes, uint32_t *status_dev, void *stream);
 
+/*
+ * cgl_get_rank_layout -- the per-rank (deduplicated) layout: a token sends ONE
+ * copy to each logical rank that hosts at least one of its experts, instead of
+ * one copy per expert.  Pages: the normal kernels' per-destination transfers
+ * and their receive counts ("All-to-All通信", the dispatch bullet: send,
+ * forward, receive per destination; caption "CPU 将隐式地等待 GPU 接收到的计数信号").
+ * Reading: this is the is_token_in_rank view of dispatch; the receiving rank
+ * then serves its local experts and returns one partial row per token.
+ *
+ * In (device): topk_idx int32 [num_tokens, num_topk] as for cgl_get_layout.
+ * Out (device, all written in full):
+ *   tokens_per_rank int32 [R]: distinct tokens reaching rank r.
+ *   rank_offset     int32 [R + 1]: exclusive prefix sum of tokens_per_rank.
+ *   max_count       int32 [1]: max over r of tokens_per_rank.
+ *   rank_dst        int32 [num_tokens, num_topk]: for the FIRST slot j of token t
+ *                   whose expert lies on rank r, the receive row of t on r; -1 for
+ *                   later slots on the same rank and for masked / out-of-range /
+ *                   over-capacity slots.
+ *   recv_token      int32 [num_tokens*num_topk] (compact) or [R*capacity] (padded):
+ *                   the source token of each receive row, -1 for rows with none.
+ * Rows of a rank hold its tokens in ascending token order.  opts.capacity > 0
+ * pads each rank to `capacity` rows (rank r at [r*capacity, ...)).
+ * Use: cgl_dispatch_fp8 / cgl_dispatch_bf16 with dst_pos = rank_dst write one
+ * copy per (token, rank); cgl_combine with dst_pos = rank_dst and unit weights
+ * sums the ranks' partial rows back in slot order.
+ * workspace: >= cgl_layout_workspace_bytes(num_tokens, num_topk, num_ranks, num_ranks)
+ *   bytes (the expert layout's size also suffices), 16-byte aligned, any contents.
+ * Errors as for cgl_get_layout.
+ */
+cgl_status cgl_get_rank_layout(const int32_t *topk_idx, int64_t num_tokens, int num_topk,
+                               int num_experts, int num_ranks, const cgl_opts *opts,
+                               int32_t *tokens_per_rank, int32_t *rank_offset, int32_t *max_count,
+                               int32_t *rank_dst, int32_t *recv_token, void *workspace,
+                               size_t workspace_bytes, uint32_t *status_dev, void *stream);
+
 /* Size of the device scratch array behind cgl_get_layout_noalloc. */
 #define CGL_NOALLOC_SCRATCH_BYTES (512u * 1024u)
 

@@ -50,6 +50,9 @@ def lib():
         L.oracle_get_layout.argtypes = [P, C.c_int64, C.c_int, C.c_int, C.c_int, C.c_int,
                                         P, P, P, P, P, P, P]
         L.oracle_get_layout.restype = C.c_int
+        L.oracle_get_rank_layout.argtypes = [P, C.c_int64, C.c_int, C.c_int, C.c_int, C.c_int,
+                                             P, P, P, P, P]
+        L.oracle_get_rank_layout.restype = C.c_int
         L.oracle_dispatch_fp8.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P, P]
         L.oracle_dispatch_fp8.restype = None
         L.oracle_dispatch_bf16.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P]
@@ -122,6 +125,33 @@ def get_layout(topk_idx: np.ndarray, num_experts: int, num_ranks: int, capacity:
     flags = lib().oracle_get_layout(_p(idx), n, k, E, R, int(capacity), _p(tpe), _p(tpr), _p(itr),
                                     _p(off), _p(mx), _p(dst), _p(src))
     return Layout(tpe, tpr, itr, off, int(mx[0]), dst, src, int(flags))
+
+
+class RankLayout(NamedTuple):
+    tokens_per_rank: np.ndarray     # int32 [R]
+    rank_offset: np.ndarray         # int32 [R + 1]
+    max_count: int
+    rank_dst: np.ndarray            # int32 [N, k]
+    recv_token: np.ndarray          # int32 [N*k] or [R*capacity]
+    flags: int
+
+
+def get_rank_layout(topk_idx: np.ndarray, num_experts: int, num_ranks: int, capacity: int = 0) -> RankLayout:
+    """Per-rank (deduplicated) layout: one row per (token, destination rank)."""
+    idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    n, k = idx.shape
+    E, R = int(num_experts), int(num_ranks)
+    if R <= 0 or E % R != 0:
+        raise ValueError("num_experts must be a positive multiple of num_ranks")
+    tpr = np.zeros(R, np.int32)
+    off = np.zeros(R + 1, np.int32)
+    mx = np.zeros(1, np.int32)
+    dst = np.zeros((n, k), np.int32)
+    rows = R * capacity if capacity > 0 else n * k
+    src = np.zeros(rows, np.int32)
+    flags = lib().oracle_get_rank_layout(_p(idx), n, k, E, R, int(capacity), _p(tpr), _p(off), _p(mx),
+                                         _p(dst), _p(src))
+    return RankLayout(tpr, off, int(mx[0]), dst, src, int(flags))
 
 
 def dispatch_fp8(x: np.ndarray, dst_pos: np.ndarray, num_rows: int):

@@ -48,3 +48,38 @@ def layout(topk_idx, num_experts: int, num_ranks: int, capacity: int = 0):
         "range_error": bad,
         "capacity_error": overflow,
     }
+
+
+def rank_layout(topk_idx, num_experts: int, num_ranks: int, capacity: int = 0):
+    """Per-rank layout, brute force: for each rank, the sorted list of tokens that
+    reach it; a token's copy for rank r is attributed to its first slot on r."""
+    n = len(topk_idx)
+    k = len(topk_idx[0]) if n else 0
+    E, R = num_experts, num_ranks
+    per = E // R
+
+    def rank_of(e):
+        return e // per if 0 <= e < E else None
+
+    tokens = {r: sorted({t for t in range(n) for j in range(k) if rank_of(topk_idx[t][j]) == r})
+              for r in range(R)}
+    counts = [len(tokens[r]) for r in range(R)]
+    offset = [sum(counts[:r]) for r in range(R + 1)]
+    rows = R * capacity if capacity > 0 else n * k
+    dst = [[-1] * k for _ in range(n)]
+    src = [-1] * rows
+    overflow = False
+    for r in range(R):
+        for slot, t in enumerate(tokens[r]):
+            j = min(j for j in range(k) if rank_of(topk_idx[t][j]) == r)
+            if capacity > 0:
+                if slot >= capacity:
+                    overflow = True
+                    continue
+                row = r * capacity + slot
+            else:
+                row = offset[r] + slot
+            dst[t][j] = row
+            src[row] = t
+    return {"tokens_per_rank": counts, "rank_offset": offset, "max_count": max(counts) if counts else 0,
+            "rank_dst": dst, "recv_token": src, "capacity_error": overflow}

@@ -196,6 +196,79 @@ int oracle_get_layout(const int32_t *topk_idx, int64_t N, int k, int E, int R, i
     return flags;
 }
 
+/*
+ * The per-rank (deduplicated) layout: a token sends one copy to each logical
+ * rank that hosts at least one of its experts, instead of one per expert.
+ * Reading: this is the DeepEP normal-mode behaviour behind "is_token_in_rank"
+ * (one transfer per token and destination rank, the rank then serves its
+ * local experts); the pages only name dispatch to experts and the host
+ * waiting on receive counts.  Rows of rank r hold its tokens in ascending
+ * token order.  rank_dst[t, j] = that row for the FIRST slot j of token t
+ * whose expert lies on rank r = e / (E/R); later slots on the same rank, and
+ * masked or out-of-range slots, get -1.  recv_token[row] = t (or -1).
+ * capacity == 0: compact rows, rank r at [rank_offset[r], rank_offset[r+1]);
+ * capacity > 0: rows [r*capacity, ...), copies past the capacity dropped and
+ * flagged.  tokens_per_rank[r] = distinct tokens reaching rank r.
+ */
+int oracle_get_rank_layout(const int32_t *topk_idx, int64_t N, int k, int E, int R, int capacity,
+                           int32_t *tokens_per_rank, int32_t *rank_offset, int32_t *max_count,
+                           int32_t *rank_dst, int32_t *recv_token) {
+    int flags = 0;
+    int per_rank = E / R;
+    int32_t first[R > 0 ? R : 1];   /* per rank: slot of its first copy in the current token */
+    for (int r = 0; r < R; ++r) tokens_per_rank[r] = 0;
+
+    /* counts: one per (token, rank) */
+    for (int64_t t = 0; t < N; ++t) {
+        for (int r = 0; r < R; ++r) first[r] = -1;
+        for (int j = 0; j < k; ++j) {
+            int32_t e = topk_idx[t * k + j];
+            if (e == -1) continue;
+            if (e < -1 || e >= E) { flags |= ORACLE_FLAG_RANGE; continue; }
+            int r = e / per_rank;
+            if (first[r] >= 0) continue;
+            first[r] = j;
+            tokens_per_rank[r] += 1;
+        }
+    }
+    rank_offset[0] = 0;
+    int32_t mx = 0;
+    for (int r = 0; r < R; ++r) {
+        rank_offset[r + 1] = rank_offset[r] + tokens_per_rank[r];
+        if (tokens_per_rank[r] > mx) mx = tokens_per_rank[r];
+    }
+    *max_count = mx;
+
+    /* rows, in token order */
+    int64_t rows = capacity > 0 ? (int64_t)R * capacity : N * k;
+    for (int64_t i = 0; i < rows; ++i) recv_token[i] = -1;
+    int32_t seen[R > 0 ? R : 1];
+    for (int r = 0; r < R; ++r) seen[r] = 0;
+    for (int64_t t = 0; t < N; ++t) {
+        for (int r = 0; r < R; ++r) first[r] = -1;
+        for (int j = 0; j < k; ++j) {
+            int32_t e = topk_idx[t * k + j];
+            int64_t p = t * k + j;
+            rank_dst[p] = -1;
+            if (e < 0 || e >= E) continue;
+            int r = e / per_rank;
+            if (first[r] >= 0) continue;
+            first[r] = j;
+            int32_t slot = seen[r]++;
+            int64_t row;
+            if (capacity > 0) {
+                if (slot >= capacity) { flags |= ORACLE_FLAG_CAPACITY; continue; }
+                row = (int64_t)r * capacity + slot;
+            } else {
+                row = rank_offset[r] + slot;
+            }
+            rank_dst[p] = (int32_t)row;
+            recv_token[row] = (int32_t)t;
+        }
+    }
+    return flags;
+}
+
 /* -------------------------------------------------------------- dispatch */
 
 /*

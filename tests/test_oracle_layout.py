@@ -129,3 +129,51 @@ def test_capacity_overflow_drops_late_tokens(oracle_mod):
     assert L.dst_pos[:, 0].tolist() == [4, 5, 6, 7, -1, -1]
     assert L.dst_pos[:, 1].tolist() == [0, 1, 2, 3, -1, -1]
     assert L.tokens_per_expert.tolist() == [6, 6, 0, 0] and L.max_count == 6
+
+
+def _compare_rank_to_brute(oracle_mod, idx, E, R, cap):
+    L = oracle_mod.get_rank_layout(idx, E, R, cap)
+    B = brute.rank_layout(idx.tolist(), E, R, cap)
+    assert L.tokens_per_rank.tolist() == B["tokens_per_rank"]
+    assert L.rank_offset.tolist() == B["rank_offset"]
+    assert L.max_count == B["max_count"]
+    assert L.rank_dst.tolist() == B["rank_dst"]
+    assert L.recv_token.tolist() == B["recv_token"]
+    assert bool(L.flags & oracle_mod.FLAG_CAPACITY) == B["capacity_error"]
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_rank_layout_brute_force(oracle_mod, seed):
+    rng = np.random.default_rng(300 + seed)
+    E = int(rng.choice([4, 8, 12, 16]))
+    R = int(rng.choice([r for r in (1, 2, 4) if E % r == 0]))
+    k = int(rng.integers(1, 6))
+    n = int(rng.integers(0, 40))
+    idx = _random_idx(rng, n, k, E, distinct=bool(seed % 2), p_bad=0.05 if seed % 3 == 0 else 0.0)
+    _compare_rank_to_brute(oracle_mod, idx, E, R, 0)
+    _compare_rank_to_brute(oracle_mod, idx, E, R, int(rng.integers(1, 12)))
+
+
+@pytest.mark.parametrize("name", W.WORKLOAD_ORDER)
+def test_rank_layout_invariants(oracle_mod, name):
+    inp = W.make_inputs(name, 0)
+    wl = inp.workload
+    E, R = wl.num_experts, wl.num_ranks
+    L = oracle_mod.get_layout(inp.topk_idx, E, R)
+    RL = oracle_mod.get_rank_layout(inp.topk_idx, E, R)
+    # same distinct-token counts as the expert layout's rank sets
+    assert np.array_equal(RL.tokens_per_rank, L.tokens_per_rank)
+    rows = int(RL.tokens_per_rank.sum())
+    used = RL.rank_dst[RL.rank_dst >= 0]
+    assert np.array_equal(np.sort(used), np.arange(rows))                 # bijection onto [0, rows)
+    tk = np.nonzero(RL.rank_dst >= 0)
+    assert np.all(RL.recv_token[RL.rank_dst[tk]] == tk[0])
+    per = E // R
+    ranks = inp.topk_idx // per
+    for t in range(0, wl.num_tokens, max(1, wl.num_tokens // 200)):   # one copy per distinct rank
+        kept = RL.rank_dst[t] >= 0
+        assert sorted(ranks[t][kept].tolist()) == sorted(set(ranks[t].tolist()))
+    for r in range(R):                                                     # ascending tokens per rank
+        seg = RL.recv_token[RL.rank_offset[r]:RL.rank_offset[r + 1]]
+        assert np.all(np.diff(seg) > 0) and np.all((ranks[seg] == r).any(axis=1))
+    assert np.all(RL.recv_token[rows:] == -1)
