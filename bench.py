@@ -180,13 +180,16 @@ def workload_label(wl: W.Workload, dedup: bool = False) -> str:
 class GpuStep:
     """Device buffers for one workload and the launch sequence of one step."""
 
-    def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False):
+    def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False, full_backward: bool = False,
+                 fused_decode: bool = False):
         import torch
 
         import combine_get_layout_02_b200 as cgl
 
         self.cgl, self.torch, self.wl, self.dev = cgl, torch, wl, device
         self.dedup = dedup
+        self.full_backward = full_backward and wl.with_grad and not dedup
+        self.fused_decode = fused_decode and wl.fp8 and not dedup
         inp = W.make_inputs(wl, seed)
         n, h, k = wl.num_tokens, wl.hidden, wl.topk
         self.host = inp
@@ -221,6 +224,7 @@ class GpuStep:
         else:
             self.recv_x = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
             self.grad_recv = torch.empty((rows, h), dtype=torch.bfloat16, device=device)
+            self.grad_w = torch.empty((n, k), dtype=torch.float32, device=device)
         self.out = torch.empty((n, h), dtype=torch.bfloat16, device=device)
         self.bytes = W.algorithmic_bytes(wl)
         if dedup:
@@ -251,6 +255,10 @@ class GpuStep:
         """(name, launches per step, algorithmic bytes per launch) of each step phase."""
         b = self.bytes
         wl = self.wl
+        if self.fused_decode:   # one launch for layout + dispatch
+            ph = [("layout+dispatch_fp8", 1, b["layout"] + b["dispatch_fp8"]),
+                  ("combine", 1, b["combine"])]
+            return ph
         if self.dedup:   # rank keys: the layout of an E = R problem
             nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_ranks, wl.num_ranks)
         else:
@@ -262,7 +270,11 @@ class GpuStep:
             ph.append(("dispatch_bf16", 1, b["dispatch_bf16"]))
         ph.append(("combine", 1, b["combine"]))
         if self.wl.with_grad:
-            ph.append(("combine_backward", 1, b["dispatch_bf16"]))
+            if self.full_backward:   # g read once, y read and grad_y written per slot, ids/weights/grad_w
+                n, h, k = wl.num_tokens, wl.hidden, wl.topk
+                ph.append(("combine_backward", 1, 2 * n * h + 4 * n * k * h + 12 * n * k))
+            else:
+                ph.append(("combine_backward", 1, b["dispatch_bf16"]))
         return ph
 
     def step_bytes(self):
@@ -274,6 +286,13 @@ class GpuStep:
         E, R = wl.num_experts, wl.num_ranks
         rec = (lambda: events.append(self._event())) if events is not None else (lambda: None)
         rec()
+        if self.fused_decode:
+            cgl.decode_dispatch_fp8(self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x,
+                                    recv_scale=self.recv_scale, status=self.status)
+            rec()
+            cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
+            rec()
+            return
         if self.dedup:
             cgl.get_rank_layout(self.idx, E, R, self.rcap, workspace=self.ws, out=self.rlay, status=self.status)
             rec()
@@ -303,8 +322,12 @@ class GpuStep:
         cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
         rec()
         if wl.with_grad:
-            cgl.dispatch_bf16(self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv,
-                              status=self.status)
+            if self.full_backward:
+                cgl.combine_backward(self.grad, self.y, self.lay.dst_pos, self.w, grad_y=self.grad_recv,
+                                     grad_w=self.grad_w, status=self.status)
+            else:
+                cgl.dispatch_bf16(self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv,
+                                  status=self.status)
             rec()
 
     def _event(self):
@@ -479,7 +502,8 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     dist_init("nccl")
     wl = W.WORKLOADS[args.workload]
-    step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup)
+    step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup, full_backward=args.full_backward,
+                   fused_decode=args.fused_decode)
     phases = step.kernels()
 
     graph = None if args.no_graph else capture_step(step)
@@ -550,7 +574,7 @@ def run_ours(args):
                          "gbs": gbs, "frac_of_peak": gbs / peak}
     dom = max(phases, key=lambda p: p[2])[0]
     src = {"combine": "combine.cu", "dispatch_fp8": "dispatch.cu", "dispatch_bf16": "dispatch.cu",
-           "layout": "layout.cu", "combine_backward": "dispatch.cu"}[dom]
+           "layout": "layout.cu", "combine_backward": "combine_backward.cu"}.get(dom, "layout.cu")
     roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
@@ -599,6 +623,10 @@ def main(argv=None):
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--dedup", action="store_true",
                     help="per-rank deduplicated dispatch: one copy per (token, rank), rank-sum combine")
+    ap.add_argument("--full-backward", action="store_true",
+                    help="bf16 workload: weighted combine backward with grad_w instead of the plain re-dispatch")
+    ap.add_argument("--fused-decode", action="store_true",
+                    help="layout and FP8 dispatch in one launch (batches of at most 1024 token-slot pairs)")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:

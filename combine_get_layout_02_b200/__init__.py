@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "CglError", "Layout", "RankLayout", "lib", "get_layout", "get_rank_layout", "dispatch_fp8", "dispatch_bf16", "combine",
-    "layout_workspace_bytes", "layout_kernel_count", "status_bits", "check_status", "new_status",
+    "combine_backward", "decode_dispatch_fp8", "layout_workspace_bytes", "layout_kernel_count", "status_bits", "check_status", "new_status",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +82,10 @@ def lib():
         L.cgl_dispatch_bf16.restype = I
         L.cgl_combine.argtypes = [P, I64, P, P, I64, I, I, P, OP, P, P]
         L.cgl_combine.restype = I
+        L.cgl_decode_dispatch_fp8.argtypes = [P, I64, I, I, I, OP, P, I, P, P, P, P, P, P, P, P, P, P, P]
+        L.cgl_decode_dispatch_fp8.restype = I
+        L.cgl_combine_backward.argtypes = [P, P, I64, P, P, I64, I, I, P, P, OP, P, P]
+        L.cgl_combine_backward.restype = I
         _lib = L
     return _lib
 
@@ -288,3 +292,61 @@ def combine(y: torch.Tensor, dst_pos: torch.Tensor, topk_weights: torch.Tensor, 
                              _opts(num_sms), _ptr(status), _stream(stream))
     _check(code, "cgl_combine")
     return out
+
+
+def combine_backward(grad_out: torch.Tensor, y: torch.Tensor, dst_pos: torch.Tensor,
+                     topk_weights: torch.Tensor, *, grad_y: Optional[torch.Tensor] = None,
+                     grad_w: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                     num_sms: int = 0, stream=None):
+    """Gradient of combine: (grad_y BF16 [rows, H], grad_w fp32 [N, k]) (cgl_combine_backward)."""
+    g = _dev(grad_out, "grad_out", torch.bfloat16, 2)
+    y = _dev(y, "y", torch.bfloat16, 2)
+    dst = _dev(dst_pos, "dst_pos", torch.int32, 2)
+    w = _dev(topk_weights, "topk_weights", torch.float32, 2)
+    n, k = dst.shape
+    h = g.shape[1]
+    if grad_y is None:
+        grad_y = torch.empty_like(y)
+    if grad_w is None:
+        grad_w = torch.empty((n, k), dtype=torch.float32, device=g.device)
+    code = lib().cgl_combine_backward(_ptr(g), _ptr(y), y.shape[0], _ptr(dst), _ptr(w), n, h, k,
+                                      _ptr(grad_y), _ptr(grad_w), _opts(num_sms), _ptr(status),
+                                      _stream(stream))
+    _check(code, "cgl_combine_backward")
+    return grad_y, grad_w
+
+
+def decode_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: int, num_ranks: int,
+                        capacity: int = 0, *, out: Optional[Layout] = None,
+                        recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
+                        status: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None):
+    """Layout + FP8 dispatch of a small (decode) batch in one launch (cgl_decode_dispatch_fp8).
+
+    Returns (Layout, recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128])."""
+    idx = _dev(topk_idx, "topk_idx", torch.int32, 2)
+    x = _dev(x, "x", torch.bfloat16, 2)
+    n, k = idx.shape
+    h = x.shape[1]
+    E, R = int(num_experts), int(num_ranks)
+    dev = idx.device
+    rows = E * capacity if capacity > 0 else n * k
+    if out is None:
+        out = Layout(
+            torch.empty(E, dtype=torch.int32, device=dev),
+            torch.empty(R, dtype=torch.int32, device=dev),
+            torch.empty((n, R), dtype=torch.uint8, device=dev),
+            torch.empty(E + 1, dtype=torch.int32, device=dev),
+            torch.empty(1, dtype=torch.int32, device=dev),
+            torch.empty((n, k), dtype=torch.int32, device=dev),
+            torch.empty(rows, dtype=torch.int32, device=dev),
+            rows, int(capacity))
+    if recv_x is None:
+        recv_x = torch.empty((rows, h), dtype=torch.uint8, device=dev)
+    if recv_scale is None:
+        recv_scale = torch.empty((rows, h // 128), dtype=torch.float32, device=dev)
+    code = lib().cgl_decode_dispatch_fp8(
+        _ptr(idx), n, k, E, R, _opts(num_sms, capacity), _ptr(x), h, _ptr(out.tokens_per_expert),
+        _ptr(out.tokens_per_rank), _ptr(out.is_token_in_rank), _ptr(out.expert_offset), _ptr(out.max_count),
+        _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(recv_x), _ptr(recv_scale), _ptr(status), _stream(stream))
+    _check(code, "cgl_decode_dispatch_fp8")
+    return out, recv_x, recv_scale

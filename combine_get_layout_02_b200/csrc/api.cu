@@ -59,6 +59,44 @@ bool ensure_smem_attr(const void *kernel, size_t bytes) {
     return true;
 }
 
+namespace {
+struct OccEntry {
+    const void *kernel;
+    int device, threads;
+    size_t smem;
+    int ctas;
+};
+OccEntry g_occ[64];
+int g_occ_n = 0;
+}  // namespace
+
+int persistent_grid(const void *kernel, int threads, size_t smem, int target_per_sm, int num_sms_cap,
+                    int64_t work) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const int sms = device_sm_count();
+    if (sms <= 0) return 0;
+    int fit = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (int i = 0; i < g_occ_n; ++i)
+            if (g_occ[i].kernel == kernel && g_occ[i].device == dev && g_occ[i].threads == threads &&
+                g_occ[i].smem == smem)
+                fit = g_occ[i].ctas;
+        if (fit == 0) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kernel, threads, smem) != cudaSuccess)
+                return 0;
+            if (fit < 1) fit = 1;
+            if (g_occ_n < 64) g_occ[g_occ_n++] = {kernel, dev, threads, smem, fit};
+        }
+    }
+    int per_sm = target_per_sm < fit ? target_per_sm : fit;
+    if (per_sm < 1) per_sm = 1;
+    const int use_sms = (num_sms_cap > 0 && num_sms_cap < sms) ? num_sms_cap : sms;
+    const int64_t want = (int64_t)use_sms * per_sm;
+    return (int)(work < want ? work : want);
+}
+
 int copy_grid(const void *kernel, int threads, int64_t work_ctas, int num_sms_cap) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -204,6 +242,48 @@ cgl_status cgl_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_
         return CGL_EALIGN;
     return launch_combine(y, recv_rows, dst_pos, topk_weights, n, h, k, out, opt_sms(opts),
                           status_dev, static_cast<cudaStream_t>(stream));
+}
+
+cgl_status cgl_combine_backward(const uint16_t *grad_out, const uint16_t *y, int64_t recv_rows,
+                                const int32_t *dst_pos, const float *topk_weights, int64_t n, int h,
+                                int k, uint16_t *grad_y, float *grad_w, const cgl_opts *opts,
+                                uint32_t *status_dev, void *stream) {
+    if (n < 0 || h <= 0 || h % 16 != 0 || h > 16384 || k < 1 || k > kMaxTopk || recv_rows < 0)
+        return CGL_EINVAL;
+    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (n > 0 && (!grad_out || !dst_pos || !topk_weights || !grad_w)) return CGL_EINVAL;
+    if (n > 0 && recv_rows > 0 && (!y || !grad_y)) return CGL_EINVAL;
+    if (!aligned(grad_out, 16) || !aligned(y, 16) || !aligned(grad_y, 16) || !aligned(dst_pos, 4) ||
+        !aligned(topk_weights, 4) || !aligned(grad_w, 4) || !aligned(status_dev, 4))
+        return CGL_EALIGN;
+    return launch_combine_backward(grad_out, y, recv_rows, dst_pos, topk_weights, n, h, k, grad_y, grad_w,
+                                   opt_sms(opts), status_dev, static_cast<cudaStream_t>(stream));
+}
+
+cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, int E, int R,
+                                   const cgl_opts *opts, const uint16_t *x, int h,
+                                   int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                                   uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
+                                   int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
+                                   float *recv_scale, uint32_t *status_dev, void *stream) {
+    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0) return CGL_EINVAL;
+    const int per_block = 1024 / k < 256 ? 1024 / k : 256;   // tokens one layout block holds
+    if (n > per_block) return CGL_EINVAL;
+    if (decode_fused_smem_bytes(n, k, E, R) > 47 * 1024) return CGL_EINVAL;
+    const int cap = opt_cap(opts);
+    if (cap < 0 || (int64_t)E * cap >= ((int64_t)1 << 31) || opt_sms(opts) < 0) return CGL_EINVAL;
+    const int64_t rows = cap > 0 ? (int64_t)E * cap : n * k;
+    if (!tokens_per_expert || !tokens_per_rank || !expert_offset || !max_count) return CGL_EINVAL;
+    if (n > 0 && (!topk_idx || !x || !dst_pos || !is_token_in_rank)) return CGL_EINVAL;
+    if (rows > 0 && (!recv_src || !recv_x || !recv_scale)) return CGL_EINVAL;
+    if (!aligned(topk_idx, 4) || !aligned(x, 16) || !aligned(tokens_per_expert, 4) ||
+        !aligned(tokens_per_rank, 4) || !aligned(is_token_in_rank, 16) || !aligned(expert_offset, 4) ||
+        !aligned(max_count, 4) || !aligned(dst_pos, 4) || !aligned(recv_src, 4) ||
+        !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(status_dev, 4))
+        return CGL_EALIGN;
+    return launch_decode_dispatch_fp8(topk_idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank,
+                                      is_token_in_rank, expert_offset, max_count, dst_pos, recv_src, recv_x,
+                                      recv_scale, opt_sms(opts), status_dev, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -28,7 +28,6 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(const uint16_t *__restrict__ y, int64_t recv_rows,
                const int32_t *__restrict__ dst_pos, const float *__restrict__ w, int64_t n, int h,
                int k, uint16_t *__restrict__ out, uint32_t *status) {
-    griddep_launch_dependents();
     griddep_wait();                   // y and dst_pos may come from the kernels just before
     const int chunks = h >> 3;
     const int64_t total = n * chunks;

@@ -34,34 +34,11 @@ constexpr int kMaxBulkHidden = 16384;    // one thread per 16 values: at most 10
 constexpr int kBulkThreadsPerSM = 1024;  // CTAs per SM of the bulk kernels = this / block size
 constexpr int kMaxBulkHiddenBf16 = 8192; // two staged BF16 rows stay within 32 KiB of shared memory
 
-__device__ __forceinline__ float absmax16(const uint4 a, const uint4 b) {
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    return m;
-}
-
-// E4M3 codes of the 16 BF16 values in (a, b), each multiplied by inv first.
-__device__ __forceinline__ uint4 quant16(const uint4 a, const uint4 b, float inv) {
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t q[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = cvt_e4m3x2(__fmul_rn(bf16_lo(w[2 * i]), inv), __fmul_rn(bf16_hi(w[2 * i]), inv));
-        const uint32_t hi =
-            cvt_e4m3x2(__fmul_rn(bf16_lo(w[2 * i + 1]), inv), __fmul_rn(bf16_hi(w[2 * i + 1]), inv));
-        q[i] = lo | (hi << 16);
-    }
-    return make_uint4(q[0], q[1], q[2], q[3]);
-}
-
 __global__ void __launch_bounds__(1024)
 dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                          const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
                          float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
     extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][h] staged code rows
-    griddep_launch_dependents();
     griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4, nblk = h >> 7;
     const int c = threadIdx.x;        // this thread's 16 values
@@ -123,7 +100,6 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                     const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
                     float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
-    griddep_launch_dependents();
     griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4;        // 16 values per thread
     const int nblk = h >> 7;          // 128-value scale blocks per row
@@ -190,7 +166,6 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
                           const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
                           int64_t recv_rows, uint32_t *status) {
     extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][2h] staged rows
-    griddep_launch_dependents();
     griddep_wait();
     const int chunks = h >> 4;
     const int c = threadIdx.x;
@@ -241,7 +216,6 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                      const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
                      int64_t recv_rows, uint32_t *status) {
-    griddep_launch_dependents();
     griddep_wait();
     const int chunks = h >> 3;        // 8 values per thread
     const int64_t total = n * chunks;
@@ -270,13 +244,9 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
     if (n * (h / 16) == 0) return CGL_OK;
     if (h <= kMaxBulkHidden) {
         const int threads = (h / 16 + 31) / 32 * 32;
-        const int sms = device_sm_count();
-        if (sms <= 0) return CGL_ECUDA;
-        const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
-        int per_sm = kBulkThreadsPerSM / threads;
-        if (per_sm < 1) per_sm = 1;
-        const int64_t want = (int64_t)use_sms * per_sm;
-        const int grid = (int)(n < want ? n : want);
+        const int grid = persistent_grid((const void *)dispatch_fp8_bulk_kernel, threads, (size_t)2 * h,
+                                         kBulkThreadsPerSM / threads, num_sms, n);
+        if (grid <= 0) return CGL_ECUDA;
         const cudaError_t err = launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)2 * h, stream, x, n, h, k, dst_pos, recv_x,
                                            recv_scale, recv_rows, status);
@@ -297,13 +267,9 @@ cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, cons
     if (n * (h / 8) == 0) return CGL_OK;
     if (h % 16 == 0 && h <= kMaxBulkHiddenBf16) {
         const int threads = (h / 16 + 31) / 32 * 32;
-        const int sms = device_sm_count();
-        if (sms <= 0) return CGL_ECUDA;
-        const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
-        int per_sm = kBulkThreadsPerSM / threads;
-        if (per_sm < 1) per_sm = 1;
-        const int64_t want = (int64_t)use_sms * per_sm;
-        const int grid = (int)(n < want ? n : want);
+        const int grid = persistent_grid((const void *)dispatch_bf16_bulk_kernel, threads, (size_t)4 * h,
+                                         kBulkThreadsPerSM / threads, num_sms, n);
+        if (grid <= 0) return CGL_ECUDA;
         const cudaError_t err = launch_pdl(dispatch_bf16_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)4 * h, stream, x, n, h, k, dst_pos, recv_x,
                                            recv_rows, status);

@@ -15,6 +15,11 @@ bool ensure_smem_attr(const void *kernel, size_t bytes);
 // SMs on the current device (cached per device); 0 on error.
 int device_sm_count();
 
+// Grid for a persistent kernel (CTAs loop over `work` items): SMs in use x
+// min(target CTAs per SM, CTAs per SM that fit), at most `work`; 0 on error.
+int persistent_grid(const void *kernel, int threads, size_t smem, int target_per_sm, int num_sms_cap,
+                    int64_t work);
+
 // Grid for a grid-stride copy kernel: enough CTAs for `work_ctas`, capped at
 // (SMs in use) x (resident CTAs per SM).
 int copy_grid(const void *kernel, int threads, int64_t work_ctas, int num_sms_cap);
@@ -69,5 +74,20 @@ cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, cons
 cgl_status launch_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_pos,
                           const float *w, int64_t n, int h, int k, uint16_t *out, int num_sms,
                           uint32_t *status, cudaStream_t stream);
+
+// Dynamic shared memory of the fused decode kernel (bytes).
+size_t decode_fused_smem_bytes(int64_t n, int k, int E, int R);
+
+cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                                      const uint16_t *x, int h, int32_t *tokens_per_expert,
+                                      int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
+                                      int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
+                                      uint8_t *recv_x, float *recv_scale, int num_sms, uint32_t *status,
+                                      cudaStream_t stream);
+
+cgl_status launch_combine_backward(const uint16_t *g, const uint16_t *y, int64_t recv_rows,
+                                   const int32_t *dst_pos, const float *w, int64_t n, int h, int k,
+                                   uint16_t *grad_y, float *grad_w, int num_sms, uint32_t *status,
+                                   cudaStream_t stream);
 
 }  // namespace cgl

@@ -163,10 +163,10 @@ __device__ __forceinline__ int pair_of(int i) { return (threadIdx.x >> 5) * (kCh
 // if an id outside [-1, E_ids) was seen (such slots make no copy).
 template <bool kRankKeys>
 __device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids, int key_div,
-                              int nkeys, const Smem &s, Pairs &P) {
+                              int nkeys, int64_t token_block, const Smem &s, Pairs &P) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int T = tokens_per_block(k);
-    P.t0 = (int64_t)blockIdx.x * T;
+    P.t0 = token_block * T;
     const int64_t rem = n - P.t0;
     P.nt = rem <= 0 ? 0 : (rem < T ? (int)rem : T);
     P.np = P.nt * k;
@@ -527,7 +527,6 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const int nb = gridDim.x, b = blockIdx.x;
     const bool with_ranks = in_rank != nullptr;
 
-    griddep_launch_dependents();   // the copy kernels may get resident; they wait for this grid
     // This launch's tag: generation + 1.  Every block reads the generation before
     // it publishes its flag, and block 0 advances it only after it has seen every
     // flag, so all blocks agree and the next launch (a graph replay too) gets a new tag.
@@ -540,7 +539,7 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     zero_words(s.hr, R);
     __syncthreads();
     Pairs P;
-    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
+    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
     if (with_ranks) rank_sets(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
@@ -594,13 +593,12 @@ layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const Smem s = carve(1, smem_count, k, E, R);
     const int tid = threadIdx.x;
     const bool with_ranks = in_rank != nullptr;
-    griddep_launch_dependents();   // the rows kernel may start; it waits for this grid
     zero_words(s.wc, kWarps * E);
     zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
     zero_words(s.hr, R);
     __syncthreads();
     Pairs P;
-    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
+    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
     if (with_ranks) rank_sets(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
@@ -625,13 +623,12 @@ layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int
     extern __shared__ __align__(16) int32_t smem_rows[];
     __shared__ int32_t scan_tmp[32];
     const Smem s = carve(2, smem_rows, k, E, R);
-    griddep_launch_dependents();   // the copy kernels may get resident; they wait for this grid
     zero_words(s.wc, kWarps * E);
     __syncthreads();
     // topk_idx is not written by the counts kernel, which started only after
     // everything before it in the stream had finished: it may be read before the wait
     Pairs P;
-    load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, s, P);
+    load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
     __syncthreads();
     warp_offsets(E, s);
     griddep_wait();
@@ -639,6 +636,122 @@ layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int
     bases_and_rows<false, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                      tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
                                      s, P, scan_tmp);
+}
+
+// Fused decode path: the layout and the FP8 dispatch of a small batch (at most
+// 1024 (token, slot) pairs) in one launch, no workspace.  Every CTA computes the
+// whole layout in shared memory (one layout block's work, so no inter-block
+// exchange), CTA 0 writes the layout outputs, and each CTA then quantises its
+// share of the tokens and writes their copies with 16-byte stores.
+__global__ void __launch_bounds__(kThreads)
+decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap,
+                    const uint16_t *__restrict__ x, int h, int32_t *__restrict__ tokens_per_expert,
+                    int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
+                    int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
+                    int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
+                    uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, uint32_t *status) {
+    extern __shared__ __align__(16) int32_t smem_decode[];
+    __shared__ int32_t scan_tmp[32];
+    const Smem s = carve(0, smem_decode, k, E, R);
+    int32_t *s_dst = smem_decode + smem_words(0, k, E, R);   // [n * k] receive row per pair
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool writer = blockIdx.x == 0;
+
+    griddep_wait();                // ids and x may come from the kernels just before
+    zero_words(s.wc, kWarps * E);
+    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
+    zero_words(s.hr, R);
+    __syncthreads();
+    Pairs P;
+    const bool bad = load_and_rank<false>(idx, n, k, E, E / R, E, 0, s, P);
+    if (writer) rank_sets(k, E, R, s, P);
+    __syncthreads();
+    warp_offsets(E, s);
+    if (writer) {
+        rank_counts(k, R, s, P);
+        write_rank_rows(R, in_rank, s, P);
+    }
+    __syncthreads();
+    const int32_t m_total = block_exclusive_scan(s.he, s.off, E, scan_tmp);
+    for (int e = tid; e < E; e += kThreads) s.base[e] = cap > 0 ? e * cap : s.off[e];
+    if (writer) {
+        int32_t mx = 0;
+        for (int e = tid; e < E; e += kThreads) {
+            tokens_per_expert[e] = s.he[e];
+            expert_offset[e] = s.off[e];
+            mx = max(mx, s.he[e]);
+        }
+        if (tid == 0) expert_offset[E] = m_total;
+        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        if (lane == 0) scan_tmp[warp] = mx;
+        __syncthreads();
+        if (tid == 0) {
+            int32_t m = 0;
+            for (int w = 0; w < kWarps; ++w) m = max(m, scan_tmp[w]);
+            *max_count = m;
+        }
+        if (cap > 0) {
+            for (int64_t i = tid; i < (int64_t)E * cap; i += kThreads) {
+                const int e = (int)(i / cap);
+                if (i - (int64_t)e * cap >= s.he[e]) recv_src[i] = -1;
+            }
+        } else {
+            for (int64_t i = m_total + tid; i < n * k; i += kThreads) recv_src[i] = -1;
+        }
+        if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
+    }
+    __syncthreads();
+    bool over = false;
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int p = pair_of(i);
+        if (p >= P.np) continue;
+        const int32_t e = P.e[i];
+        int32_t d = -1;
+        if (e >= 0) {
+            const int32_t pos = s.base[e] + s.wc[warp * E + e] + P.rk[i];
+            if (cap > 0 && pos - e * cap >= cap) over = true;
+            else if (pos < recv_rows) d = pos;
+        }
+        s_dst[p] = d;
+        if (writer) {
+            dst_pos[p] = d;
+            if (d >= 0) recv_src[d] = p;
+        }
+    }
+    if (writer && over) report(status, kErrCapacity);
+    __syncthreads();
+
+    // dispatch this CTA's tokens: 16 values per thread per pass, 8 lanes per scale block
+    const int chunks = h >> 4, nblk = h >> 7;
+    for (int64_t t = blockIdx.x; t < n; t += gridDim.x) {
+        for (int c0 = warp * 32; c0 < chunks; c0 += kThreads) {   // warp-uniform
+            const int c = c0 + lane;
+            const bool active = c < chunks;
+            uint4 a = make_uint4(0, 0, 0, 0), b = a;
+            if (active) {
+                a = ld_nc_v4(x + t * h + (int64_t)c * 16);
+                b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
+            }
+            float m = absmax16(a, b);
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            if (!active) continue;
+            const float amax_c = fmaxf(m, 1e-4f);
+            const float scale = __fdiv_rn(amax_c, 448.0f);
+            const float inv = __fdiv_rn(448.0f, amax_c);
+            const uint4 q = quant16(a, b, inv);
+            for (int j = 0; j < k; ++j) {
+                const int32_t row = s_dst[t * k + j];
+                if (row < 0) continue;
+                st_cs_v4(recv_x + (int64_t)row * h + (int64_t)c * 16, q);
+                if ((c & 7) == 0) recv_scale[(int64_t)row * nblk + (c >> 3)] = scale;
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -742,6 +855,28 @@ cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R
                               cudaStream_t stream) {
     return launch_layout_impl<true>(idx, n, k, E, R, cap, tokens_per_rank, nullptr, nullptr, rank_offset,
                                     max_count, rank_dst, recv_token, ws, status, stream);
+}
+
+size_t decode_fused_smem_bytes(int64_t n, int k, int E, int R) {
+    return (smem_words(0, k, E, R) + (size_t)(n * k)) * sizeof(int32_t);
+}
+
+cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                                      const uint16_t *x, int h, int32_t *tokens_per_expert,
+                                      int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
+                                      int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
+                                      uint8_t *recv_x, float *recv_scale, int num_sms, uint32_t *status,
+                                      cudaStream_t stream) {
+    const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
+    const int sms = device_sm_count();
+    if (sms <= 0) return CGL_ECUDA;
+    const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+    const int64_t grid = n < 1 ? 1 : (n < use_sms ? n : use_sms);
+    const cudaError_t err = launch_pdl(decode_fused_kernel, dim3((unsigned)grid), dim3(kThreads),
+                                       decode_fused_smem_bytes(n, k, E, R), stream, idx, n, k, E, R, cap, x, h,
+                                       tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
+                                       dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 }  // namespace cgl

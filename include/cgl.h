@@ -261,6 +261,54 @@ cgl_status cgl_combine(const uint16_t *y, int64_t num_recv_rows, const int32_t *
                        const float *topk_weights, int64_t num_tokens, int hidden, int num_topk,
                        uint16_t *out, const cgl_opts *opts, uint32_t *status_dev, void *stream);
 
+/*
+ * cgl_decode_dispatch_fp8 -- the decode path in one launch: cgl_get_layout and
+ * cgl_dispatch_fp8 fused for a small batch, with no workspace.  Pages: the
+ * low-latency kernels for decoding (news article feature list and
+ * "具体性能方面": 128 tokens per batch, hidden 7168, top-8, FP8 dispatch, BF16
+ * combine; brainleap "Pure RDMA 的低延迟内核"), here on one GPU: one launch
+ * instead of two, no device-to-host count read when opts.capacity fixes the
+ * per-expert capacity in advance (what a captured CUDA graph needs).
+ * Same outputs, ordering and errors as cgl_get_layout followed by
+ * cgl_dispatch_fp8 with the layout's dst_pos (receive rows = E*capacity when
+ * opts.capacity > 0, else num_tokens*num_topk; rows past a full expert are
+ * dropped with CGL_ECAPACITY).
+ * Limits (CGL_EINVAL otherwise): num_tokens <= min(256, 1024 / num_topk)
+ * (128 at top-8); hidden % 128 == 0; the shared memory the kernel needs
+ * (per-block counts for E experts, the batch's (token, slot) rows) within
+ * 47 KiB.  opts.num_sms caps the grid (one CTA per token otherwise).
+ * Alignment: x, recv_x and is_token_in_rank 16-byte aligned; int32/fp32 arrays 4-byte.
+ */
+cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t num_tokens, int num_topk,
+                                   int num_experts, int num_ranks, const cgl_opts *opts,
+                                   const uint16_t *x, int hidden, int32_t *tokens_per_expert,
+                                   int32_t *tokens_per_rank, uint8_t *is_token_in_rank,
+                                   int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
+                                   int32_t *recv_src, uint8_t *recv_x, float *recv_scale,
+                                   uint32_t *status_dev, void *stream);
+
+/*
+ * cgl_combine_backward -- the gradient of cgl_combine.  Pages: combine
+ * accumulates the experts' outputs (brainleap "Day2 DeepEP", "All-to-All通信");
+ * this is its derivative for training.  For an output gradient g = dL/dout:
+ *   grad_y[dst_pos[t, j], h] = bf16_rn( w[t, j] * g[t, h] )   (one binary32 product)
+ *   grad_w[t, j]             = sum_h g[t, h] * y[dst_pos[t, j], h]   (binary32)
+ * grad_w's summation order is this library's (per-thread fused multiply-adds,
+ * then a fixed tree over the block): deterministic, within a few binary32
+ * roundings of the exact sum; slots with dst_pos < 0 give grad_w = 0 and write
+ * no row.
+ * In (device): grad_out BF16 [num_tokens, hidden]; y BF16 [num_recv_rows, hidden]
+ *   (the expert outputs combine read); dst_pos, topk_weights as for cgl_combine.
+ * Out (device): grad_y BF16 [num_recv_rows, hidden] (rows with no slot untouched);
+ *   grad_w fp32 [num_tokens, num_topk] (every element written).
+ * Requires hidden % 16 == 0 and hidden <= 16384; grad_out, y, grad_y 16-byte aligned.
+ * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows (that slot is skipped).
+ */
+cgl_status cgl_combine_backward(const uint16_t *grad_out, const uint16_t *y, int64_t num_recv_rows,
+                                const int32_t *dst_pos, const float *topk_weights, int64_t num_tokens,
+                                int hidden, int num_topk, uint16_t *grad_y, float *grad_w,
+                                const cgl_opts *opts, uint32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -57,6 +57,8 @@ def lib():
         L.oracle_dispatch_fp8.restype = None
         L.oracle_dispatch_bf16.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P]
         L.oracle_dispatch_bf16.restype = None
+        L.oracle_combine_backward.argtypes = [P, P, P, P, C.c_int64, C.c_int, C.c_int, P, P]
+        L.oracle_combine_backward.restype = None
         L.oracle_combine.argtypes = [P, P, P, C.c_int64, C.c_int, C.c_int, P]
         L.oracle_combine.restype = None
         _lib = L
@@ -189,3 +191,17 @@ def combine(y: np.ndarray, dst_pos: np.ndarray, topk_w: np.ndarray) -> np.ndarra
     out = np.zeros((n, h), np.uint16)
     lib().oracle_combine(_p(y), _p(dst), _p(w), n, h, k, _p(out))
     return out
+
+
+def combine_backward(g: np.ndarray, y: np.ndarray, dst_pos: np.ndarray, topk_w: np.ndarray):
+    """Returns (grad_y uint16 [rows, H], grad_w fp32 [N, k]); rows with no slot are zero."""
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    y = np.ascontiguousarray(y, dtype=np.uint16)
+    dst = np.ascontiguousarray(dst_pos, dtype=np.int32)
+    w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    n, k = dst.shape
+    h = g.shape[1]
+    gy = np.zeros(y.shape, np.uint16)
+    gw = np.zeros((n, k), np.float32)
+    lib().oracle_combine_backward(_p(g), _p(y), _p(dst), _p(w), n, h, k, _p(gy), _p(gw))
+    return gy, gw

@@ -348,3 +348,36 @@ void oracle_combine(const uint16_t *y, const int32_t *dst_pos, const float *topk
             out[t * H + h] = oracle_bf16_from_f32(acc);
         }
 }
+
+/* ------------------------------------------------------- combine backward */
+
+/*
+ * Backward of combine (out[t] = sum_j w[t,j] * y[dst_pos[t,j]]) for an output
+ * gradient g = dL/dout, BF16 [N, H]:
+ *   grad_y[dst_pos[t,j], h] = bf16( w[t,j] * g[t,h] )   (one binary32 product, RNE)
+ *   grad_w[t, j] = sum_h g[t,h] * y[dst_pos[t,j], h]     (accumulated in double, then
+ *                                                          rounded once to binary32)
+ * Slots with dst_pos < 0 write no row and get grad_w = 0.  Reading: the pages
+ * only say that combine accumulates; this is its derivative, with the weight
+ * gradient's reduction order left free (hence the double accumulation here:
+ * the exact value up to one final rounding).
+ */
+void oracle_combine_backward(const uint16_t *g, const uint16_t *y, const int32_t *dst_pos,
+                             const float *topk_w, int64_t N, int H, int k, uint16_t *grad_y,
+                             float *grad_w) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t)
+        for (int j = 0; j < k; ++j) {
+            int32_t row = dst_pos[t * k + j];
+            if (row < 0) { grad_w[t * k + j] = 0.0f; continue; }
+            float w = topk_w[t * k + j];
+            double dot = 0.0;
+            for (int h = 0; h < H; ++h) {
+                float gv = bf16_to_f32(g[t * H + h]);
+                float prod = w * gv;
+                grad_y[(int64_t)row * H + h] = oracle_bf16_from_f32(prod);
+                dot += (double)gv * (double)bf16_to_f32(y[(int64_t)row * H + h]);
+            }
+            grad_w[t * k + j] = (float)dot;
+        }
+}

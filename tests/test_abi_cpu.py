@@ -111,3 +111,34 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(TypeError):
         cgl.combine(torch.zeros(8, 8, dtype=torch.bfloat16), torch.zeros(1, 8, dtype=torch.int32),
                     torch.zeros(1, 8))
+
+
+def test_combine_backward_host_errors(L):
+    p = FAKE
+    assert L.cgl_combine_backward(p, p, 128, p, p, 16, 7160, 8, p, p, None, None, None) == cgl.EINVAL   # H % 16
+    assert L.cgl_combine_backward(p, p, 128, p, p, 16, 16400, 8, p, p, None, None, None) == cgl.EINVAL  # H > 16384
+    assert L.cgl_combine_backward(p, p, 128, p, p, 16, 7168, 8, p, None, None, None, None) == cgl.EINVAL
+    assert L.cgl_combine_backward(p, p + 8, 128, p, p, 16, 7168, 8, p, p, None, None, None) == cgl.EALIGN
+    assert L.cgl_combine_backward(p, p, 128, p, p, 16, 7168, 8, p + 4, p, None, None, None) == cgl.EALIGN
+
+
+def test_rank_layout_host_errors(L):
+    p = FAKE
+    ws = L.cgl_layout_workspace_bytes(128, 8, 64, 64)
+    call = lambda **kw: L.cgl_get_rank_layout(kw.get("idx", p), 128, 8, 256, kw.get("R", 64), None, p, p, p,
+                                              kw.get("dst", p), p, kw.get("ws", p), kw.get("wsb", ws), None, None)
+    assert call(R=60) == cgl.EINVAL
+    assert call(wsb=ws - 1) == cgl.EINVAL
+    assert call(dst=None) == cgl.EINVAL
+    assert call(ws=p + 8) == cgl.EALIGN
+    assert call(idx=p + 2) == cgl.EALIGN
+
+
+def test_decode_dispatch_host_errors(L):
+    p = FAKE
+    o = lambda cap=0, sms=0: C.byref(cgl.Opts(sms, cap))
+    args = lambda n=128, k=8, h=7168, x=p, itr=p: (p, n, k, 256, 32, o(), x, h, p, p, itr, p, p, p, p, p, p, None, None)
+    assert L.cgl_decode_dispatch_fp8(*args(n=129)) == cgl.EINVAL        # more than one layout block at k = 8
+    assert L.cgl_decode_dispatch_fp8(*args(h=7000)) == cgl.EINVAL       # hidden % 128
+    assert L.cgl_decode_dispatch_fp8(*args(x=p + 8)) == cgl.EALIGN
+    assert L.cgl_decode_dispatch_fp8(*args(itr=p + 4)) == cgl.EALIGN
