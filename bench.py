@@ -42,9 +42,9 @@ FALLBACK_HBM_GBS = 6650.0
 # for the kernels at the 4096-token prefill shape, with the sha256 of the kernel
 # source they were taken on; a changed source reports traffic null.
 NCU_TRAFFIC = {
-    "combine": {"bytes": 506999296, "src_sha": "b4d10dad3865f683"},
-    "dispatch_fp8": {"bytes": 242101248, "src_sha": "12e36f8c2e7dbd8e"},
-    "layout": {"bytes": 198400, "src_sha": "041e4a9928bdb3da"},
+    "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
+    "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
+    "layout": {"bytes": 210176, "src_sha": "55a9ef26e30253f8"},
 }
 
 
@@ -502,6 +502,10 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     dist_init("nccl")
     wl = W.WORKLOADS[args.workload]
+    if args.num_tokens:
+        import dataclasses
+
+        wl = dataclasses.replace(wl, num_tokens=args.num_tokens)
     step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup, full_backward=args.full_backward,
                    fused_decode=args.fused_decode)
     phases = step.kernels()
@@ -616,6 +620,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=W.WORKLOAD_ORDER, default="prefill")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--num-tokens", type=int, default=0,
+                    help="override the workload's token count (e.g. small cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
