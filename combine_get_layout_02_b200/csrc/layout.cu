@@ -503,6 +503,35 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
     if (bad_row) report(status, kErrRange);
 }
 
+// Wait until flags[0..nb) all hold `tag` (acquire), polling one flag per
+// thread at a time, for at most kWaitCycles (~1 s).  Returns true for the
+// whole block when every flag was seen; otherwise reports CGL_ETIMEOUT and
+// returns false for the whole block.  All threads of the block must call it.
+__device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint32_t *status) {
+    bool timed_out = false;
+    const long long start = clock64();
+    for (int bb = threadIdx.x; bb < nb && !timed_out; bb += kThreads) {
+        while (ld_acquire_u64(flags + bb) != tag) {
+            if (clock64() - start > kWaitCycles) { timed_out = true; break; }
+            __nanosleep(64);
+        }
+    }
+    __threadfence();
+    if (__syncthreads_or(timed_out)) {
+        if (threadIdx.x == 0) report(status, 1u << CGL_ETIMEOUT);
+        return false;
+    }
+    return true;
+}
+
+// Self-test of the bounded wait: one block waits for flags that hold a tag no
+// kernel writes (kTagHigh | 0, generation 0 is never a launch's tag), so it
+// must give up after ~1 s and report CGL_ETIMEOUT.
+__global__ void __launch_bounds__(kThreads) wait_probe_kernel(const uint64_t *flags, int nflags,
+                                                              uint32_t *status) {
+    wait_for_flags(flags, nflags, kTagHigh, status);
+}
+
 __device__ void zero_words(int32_t *p, int n) {
     for (int i = threadIdx.x; i < n; i += kThreads) p[i] = 0;
 }
@@ -565,19 +594,7 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     }
 
     // every block's counts must be visible before the bases
-    bool timed_out = false;
-    const long long start = clock64();
-    for (int bb = tid; bb < nb && !timed_out; bb += kThreads) {
-        while (ld_acquire_u64(flags + bb) != tag) {
-            if (clock64() - start > kWaitCycles) { timed_out = true; break; }
-            __nanosleep(64);
-        }
-    }
-    __threadfence();
-    if (__syncthreads_or(timed_out)) {
-        if (tid == 0) report(status, 1u << CGL_ETIMEOUT);
-        return;
-    }
+    if (!wait_for_flags(flags, nb, tag, status)) return;
     if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
     bases_and_rows<true, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                     tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
@@ -855,6 +872,11 @@ cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R
                               cudaStream_t stream) {
     return launch_layout_impl<true>(idx, n, k, E, R, cap, tokens_per_rank, nullptr, nullptr, rank_offset,
                                     max_count, rank_dst, recv_token, ws, status, stream);
+}
+
+cgl_status launch_wait_probe(const uint64_t *flags, int nflags, uint32_t *status, cudaStream_t stream) {
+    wait_probe_kernel<<<1, kThreads, 0, stream>>>(flags, nflags, status);
+    return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 size_t decode_fused_smem_bytes(int64_t n, int k, int E, int R) {

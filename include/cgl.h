@@ -309,6 +309,18 @@ cgl_status cgl_combine_backward(const uint16_t *grad_out, const uint16_t *y, int
                                 int hidden, int num_topk, uint16_t *grad_y, float *grad_w,
                                 const cgl_opts *opts, uint32_t *status_dev, void *stream);
 
+/*
+ * cgl_selftest_bounded_wait -- diagnostic for failure detection.  Runs the
+ * layout's inter-block wait (the only wait in any kernel of this library) in
+ * one block, on `nflags` device words that no kernel writes with the tag it
+ * waits for.  The wait must give up after ~1 s (2^31 SM cycles), OR
+ * 1u << CGL_ETIMEOUT into *status_dev and return; the stream and the context
+ * stay usable.  flags: device, 8-byte aligned, nflags in [1, 4096], any
+ * contents (zeroed memory works).  The pages have no counterpart.
+ */
+cgl_status cgl_selftest_bounded_wait(const uint64_t *flags, int nflags, uint32_t *status_dev,
+                                     void *stream);
+
 #ifdef __cplusplus
 }
 #endif
