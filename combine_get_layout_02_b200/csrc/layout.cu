@@ -7,22 +7,30 @@
 // an expert is ascending token order: the result equals one sequential walk
 // over t = 0..N-1, j = 0..k-1 that hands out the next free row of each expert.
 //
-// Work split.  Block b owns T consecutive tokens, T = min(256, 1024 / k), so
-// at most 1024 (token, slot) pairs; pair p of the block (row-major (t, j)
-// order) belongs to warp p / 128, which walks its 4 chunks of 32 pairs in order.
+// Work split.  Block b owns T consecutive tokens, T = min(64 CH, 256 CH / k),
+// so at most 256 CH (token, slot) pairs, CH = 1, 2 or 4 chunks of 32 pairs per
+// warp; pair p of the block (row-major (t, j) order) belongs to warp
+// p / (32 CH), which walks its chunks in order.  The whole layout is latency
+// bound: every phase is a few instructions per pair on one SM, so the pairs
+// are spread over more blocks (smaller CH) until the grid reaches 64 blocks;
+// past that the all-blocks read of the count table (blocks^2 (E + R) words
+// through L2) costs more than the per-pair work it saves.
 //
 //   ranks in warp : per chunk, __match_any_sync groups the lanes that name
 //                   one expert; a lane's rank is the warp's running count of
 //                   that expert plus the lower lanes of its group, and the
 //                   group's lowest lane advances the count (warp-private
 //                   shared-memory counters, one per expert).  A token that
-//                   names one expert twice needs no special case.
+//                   names one expert twice needs no special case.  (On
+//                   sm_100a match.any costs ~390 cycles of latency and ~56
+//                   SM cycles of issue per warp: the main per-pair cost.)
 //   block counts  : a per-expert pass over the 8 warps turns the warp counts
 //                   into warp offsets and the block's count per expert.
 //   rank sets     : per token, the set of ranks it reaches (slots of one
 //                   token are adjacent lanes: a segmented shuffle-OR when k
 //                   divides 32, shared-memory atomics otherwise); distinct
-//                   tokens per rank come from ballots; the bitmasks are
+//                   tokens per rank come from ballots (idle warps split
+//                   the ranks); the bitmasks are
 //                   expanded to the block's is_token_in_rank bytes with
 //                   coalesced 16-byte stores.
 //   bases         : every block reads the workspace table of per-block counts
@@ -38,7 +46,10 @@
 // everything and the blocks exchange their counts through the workspace: each
 // block writes its row, then release-stores this launch's 64-bit tag into its
 // flag word, and waits, with a bounded spin (CGL_ETIMEOUT after ~1 s), until
-// every flag shows that tag.  The tag is a generation counter kept in the
+// every flag shows that tag; one warp polls with relaxed loads and a single
+// fence follows (an acquire load per poll would invalidate L1 every time).
+// One exchange round only: on this part each dependent round trip through L2
+// costs about a microsecond, more than the column sums it would save.  The tag is a generation counter kept in the
 // workspace (+1 per launch), so it changes on every launch, replays of a
 // captured graph included.  Otherwise two kernels run (counts, then bases +
 // rows), the second with programmatic dependent launch; it recomputes the
@@ -63,9 +74,24 @@ constexpr size_t kSmemDefault = 47 * 1024;        // dynamic bytes that need no 
                                                   // minus room for static shared memory)
 constexpr long long kWaitCycles = 1LL << 31;      // bound on the inter-block wait (~1 s)
 
-__host__ __device__ __forceinline__ int tokens_per_block(int k) {
-    const int t = kMaxPairs / k;
-    return t < kMaxTokensPerBlock ? (t > 0 ? t : 1) : kMaxTokensPerBlock;
+// Tokens per block when each warp takes CH chunks of 32 pairs (CH = 1, 2, 4).
+__host__ __device__ __forceinline__ int tokens_per_block(int k, int CH = kChunks) {
+    const int t = (kThreads * CH) / k;
+    const int cap = kMaxTokensPerBlock / kChunks * CH;
+    return t < cap ? (t > 0 ? t : 1) : cap;
+}
+
+// Chunks per warp of the one-launch layout for n tokens: a single block when
+// all pairs fit in one, else the smallest of 1, 2, 4 that keeps the grid at
+// most kSpreadBlocks blocks (fewer pairs per SM, same number of exchange rows).
+constexpr int kSpreadBlocks = 64;
+__host__ __device__ __forceinline__ int layout_chunks(int64_t n, int k) {
+    if (n <= tokens_per_block(k, kChunks)) return kChunks;
+    for (int ch = 1; ch < kChunks; ch *= 2) {
+        const int t = tokens_per_block(k, ch);
+        if ((n + t - 1) / t <= kSpreadBlocks) return ch;
+    }
+    return kChunks;
 }
 __host__ __device__ __forceinline__ int mask_words(int R) { return (R + 31) >> 5; }
 
@@ -80,7 +106,7 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 WsLayout ws_layout(int64_t n, int k, int E, int R) {
     WsLayout w;
-    const int T = tokens_per_block(k);
+    const int T = tokens_per_block(k, layout_chunks(n, k));
     w.blocks = n > 0 ? (n + T - 1) / T : 1;
     w.e_off = align256((size_t)(w.blocks + 1) * sizeof(uint64_t));
     w.r_off = w.e_off + align256((size_t)w.blocks * (size_t)E * sizeof(int32_t));
@@ -102,11 +128,11 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
 // Flags hold this constant in their high half; counts (non-negative int32) never do.
 constexpr uint64_t kTagHigh = 0x9E3779B9ull << 32;
 
-__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
-    uint64_t v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
+
+// q = e / d for 0 <= e < 1024 and 1 <= d <= 1024 as (e * m) >> 20 with
+// m = ceil(2^20 / d): exact on that range because e * (m * d - 2^20) < 2^20.
+__device__ __forceinline__ uint32_t div_magic(int d) { return ((1u << 20) + (uint32_t)d - 1u) / (uint32_t)d; }
+__device__ __forceinline__ int div_small(int e, uint32_t m) { return (int)(((uint32_t)e * m) >> 20); }
 
 // Shared memory (32-bit words).  kind 0: fused kernel, 1: counts kernel, 2: rows kernel.
 struct Smem {
@@ -144,28 +170,27 @@ __device__ Smem carve(int kind, int32_t *p, int k, int E, int R) {
     return s;
 }
 
-// Block-level view of one block's pairs.
-struct Pairs {
+// Block-level view of one block's pairs; CH = 32-pair chunks per warp (a block
+// holds up to 8 * 32 * CH pairs).
+template <int CH>
+struct PairsT {
     int64_t t0;      // first token of the block
     int nt;          // tokens in the block
     int np;          // pairs in the block (nt * k)
-    int32_t e[kChunks];    // expert of each of this thread's pairs (-1: no copy)
-    int32_t rk[kChunks];   // rank among the warp's earlier pairs of that expert
+    int32_t e[CH];   // key of each of this thread's pairs (-1: no copy)
+    int32_t rk[CH];  // rank among the warp's earlier pairs with that key
 };
+using Pairs = PairsT<kChunks>;
 
-__device__ __forceinline__ int pair_of(int i) { return (threadIdx.x >> 5) * (kChunks * 32) + i * 32 + (threadIdx.x & 31); }
+template <int CH = kChunks>
+__device__ __forceinline__ int pair_of(int i) { return (threadIdx.x >> 5) * (CH * 32) + i * 32 + (threadIdx.x & 31); }
 
 // Load this thread's ids (coalesced: each warp reads 32 consecutive ids per
-// chunk), turn them into keys and rank the keys within the warp.  Expert mode:
-// key = expert id.  Rank mode (kRankKeys): key = the expert's rank e / key_div
-// for the first slot of the token on that rank, else -1 (one copy per token
-// and rank).  Keys index s.wc[.][0, nkeys).  s.wc must be zero.  Returns true
-// if an id outside [-1, E_ids) was seen (such slots make no copy).
-template <bool kRankKeys>
-__device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids, int key_div,
-                              int nkeys, int64_t token_block, const Smem &s, Pairs &P) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int T = tokens_per_block(k);
+// chunk) of block `token_block` (T tokens per block).  Returns true if an id
+// outside [-1, E_ids) was seen (such slots make no copy).
+template <int CH = kChunks>
+__device__ __forceinline__ bool load_pairs(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids,
+                                           int64_t token_block, int T, PairsT<CH> &P) {
     P.t0 = token_block * T;
     const int64_t rem = n - P.t0;
     P.nt = rem <= 0 ? 0 : (rem < T ? (int)rem : T);
@@ -173,34 +198,61 @@ __device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k,
     const int32_t *src = idx + P.t0 * k;
     bool bad = false;
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int p = pair_of(i);
+    for (int i = 0; i < CH; ++i) {
+        const int p = pair_of<CH>(i);
         P.e[i] = p < P.np ? __ldg(src + p) : -1;
     }
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
+    for (int i = 0; i < CH; ++i) {
         if (P.e[i] < -1 || P.e[i] >= E_ids) { bad = true; P.e[i] = -1; }
     }
+    return bad;
+}
+
+// Turn the loaded ids into keys and rank the keys within the warp.  Expert
+// mode: key = expert id.  Rank mode (kRankKeys): key = the expert's rank
+// e / key_div for the first slot of the token on that rank, else -1 (one copy
+// per token and rank).  Keys index s.wc[.][0, nkeys).  s.wc must be zero.
+template <bool kRankKeys, int CH = kChunks>
+__device__ __forceinline__ void key_and_rank(const int32_t *__restrict__ idx, int k, int E_ids, int key_div,
+                                             int nkeys, const Smem &s, PairsT<CH> &P) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lower = (1u << lane) - 1u;
     if (kRankKeys) {
+        const uint32_t m = div_magic(key_div);
+        if ((32 % k) == 0) {
+            // a token's slots are adjacent lanes of one chunk: the first slot on a
+            // rank is the lowest lane of its (token, rank) group
+            const int tshift = __ffs(k) - 1;
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) {
-            const int32_t e = P.e[i];
-            if (e < 0) continue;
-            const int p = pair_of(i);
-            const int tl = p / k, j = p - tl * k;
-            const int r = e / key_div;
-            bool first = true;
-            for (int jj = 0; jj < j; ++jj) {
-                const int32_t e2 = __ldg(src + tl * k + jj);
-                if (e2 >= 0 && e2 < E_ids && e2 / key_div == r) first = false;
+            for (int i = 0; i < CH; ++i) {
+                const int32_t e = P.e[i];
+                const int r = e >= 0 ? div_small(e, m) : 0;
+                const int key = e >= 0 ? (((lane >> tshift) << 11) | r) : (int)(0x80000000u | (uint32_t)lane);
+                const unsigned grp = __match_any_sync(0xFFFFFFFFu, key);
+                P.e[i] = (e >= 0 && (grp & lower) == 0) ? r : -1;
             }
-            P.e[i] = first ? r : -1;
+        } else {
+            const int32_t *src = idx + P.t0 * k;
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                const int32_t e = P.e[i];
+                if (e < 0) continue;
+                const int p = pair_of<CH>(i);
+                const int tl = p / k, j = p - tl * k;
+                const int r = div_small(e, m);
+                bool first = true;
+                for (int jj = 0; jj < j; ++jj) {
+                    const int32_t e2 = __ldg(src + tl * k + jj);
+                    if (e2 >= 0 && e2 < E_ids && div_small(e2, m) == r) first = false;
+                }
+                P.e[i] = first ? r : -1;
+            }
         }
     }
     int32_t *wc = s.wc + warp * nkeys;
-    const uint32_t lower = (1u << lane) - 1u;
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
+    for (int i = 0; i < CH; ++i) {
         const int32_t e = P.e[i];
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
         const int32_t before = e >= 0 ? wc[e] : 0;
@@ -209,15 +261,23 @@ __device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k,
         __syncwarp();
         P.rk[i] = before + __popc(peers & lower);
     }
+}
+
+template <bool kRankKeys, int CH = kChunks>
+__device__ bool load_and_rank(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids, int key_div,
+                              int nkeys, int64_t token_block, int T, const Smem &s, PairsT<CH> &P) {
+    const bool bad = load_pairs<CH>(idx, n, k, E_ids, token_block, T, P);
+    key_and_rank<kRankKeys, CH>(idx, k, E_ids, key_div, nkeys, s, P);
     return bad;
 }
 
 // Warp counts -> warp offsets (in place) and block counts per expert.  Needs a barrier before.
+template <int NT = kThreads>
 __device__ void warp_offsets(int E, const Smem &s) {
-    for (int e = threadIdx.x; e < E; e += kThreads) {
+    for (int e = threadIdx.x; e < E; e += NT) {
         int32_t run = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < (NT / 32); ++w) {
             const int32_t c = s.wc[w * E + e];
             s.wc[w * E + e] = run;
             run += c;
@@ -227,18 +287,21 @@ __device__ void warp_offsets(int E, const Smem &s) {
 }
 
 // Rank sets of the block's tokens into s.mask (zeroed before).
-__device__ void rank_sets(int k, int E, int R, const Smem &s, const Pairs &P) {
+template <int CH = kChunks>
+__device__ void rank_sets(int k, int E, int R, const Smem &s, const PairsT<CH> &P) {
     const int lane = threadIdx.x & 31;
-    const int per = E / R;
+    const uint32_t pm = div_magic(E / R);
     const int rw = mask_words(R);
     if ((32 % k) == 0 && R <= 64) {
         // the k slots of a token are k adjacent lanes of one chunk
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) {
+        for (int i = 0; i < CH; ++i) {
             const int32_t e = P.e[i];
-            uint64_t m = e >= 0 ? (1ull << (e / per)) : 0ull;
-            for (int o = 1; o < k; o <<= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
-            const int p = pair_of(i);
+            uint64_t m = e >= 0 ? (1ull << div_small(e, pm)) : 0ull;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1)
+                if (o < k) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
+            const int p = pair_of<CH>(i);
             if (p < P.np && (lane % k) == 0) {
                 const int tl = p / k;
                 s.mask[tl * rw] = (uint32_t)m;
@@ -247,39 +310,50 @@ __device__ void rank_sets(int k, int E, int R, const Smem &s, const Pairs &P) {
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) {
+        for (int i = 0; i < CH; ++i) {
             const int32_t e = P.e[i];
             if (e < 0) continue;
-            const int r = e / per;
-            atomicOr(&s.mask[(pair_of(i) / k) * rw + (r >> 5)], 1u << (r & 31));
+            const int r = div_small(e, pm);
+            atomicOr(&s.mask[(pair_of<CH>(i) / k) * rw + (r >> 5)], 1u << (r & 31));
         }
     }
 }
 
-// Distinct tokens per rank of the block into s.hr (zeroed before).  Needs a barrier before.
-__device__ void rank_counts(int k, int R, const Smem &s, const Pairs &P) {
+// Distinct tokens per rank of the block into s.hr (zeroed before).  Needs a
+// barrier before.  R <= 64: one ballot per (32-token group, rank); when there
+// are more warps than token groups, the spare warps split the ranks.
+template <int CH = kChunks, int NT = kThreads>
+__device__ void rank_counts(int k, int R, const Smem &s, const PairsT<CH> &P) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int rw = mask_words(R);
     if (R <= 64) {
-        // warp w counts tokens [32 w', 32 w' + 32) for w' = w, w + 8, ...: one ballot per rank
-        for (int tb = warp * 32; tb < P.nt; tb += kThreads) {
-            const int tl = tb + lane;
+        constexpr int kW = NT / 32;
+        const int ngroups = (P.nt + 31) >> 5;
+        if (ngroups == 0) return;
+        const int slices = ngroups >= kW ? 1 : kW / ngroups;
+        const int slice = warp / (ngroups >= kW ? kW : ngroups);
+        if (slice >= slices) return;
+        const int r0 = R * slice / slices, r1 = R * (slice + 1) / slices;
+        const int g0 = ngroups >= kW ? warp : warp % ngroups;
+        const int gstep = ngroups >= kW ? kW : ngroups;
+        for (int g = g0; g < ngroups; g += gstep) {
+            const int tl = g * 32 + lane;
             uint64_t m = 0;
             if (tl < P.nt) {
                 m = s.mask[tl * rw];
                 if (rw > 1) m |= (uint64_t)s.mask[tl * rw + 1] << 32;
             }
             int32_t c0 = 0, c1 = 0;
-            for (int r = 0; r < R; ++r) {
+            for (int r = r0; r < r1; ++r) {
                 const int c = __popc(__ballot_sync(0xFFFFFFFFu, (m >> r) & 1ull));
                 if (r == lane) c0 = c;
                 if (r == lane + 32) c1 = c;
             }
-            if (lane < R && c0) atomicAdd(&s.hr[lane], c0);
-            if (lane + 32 < R && c1) atomicAdd(&s.hr[lane + 32], c1);
+            if (c0) atomicAdd(&s.hr[lane], c0);
+            if (c1) atomicAdd(&s.hr[lane + 32], c1);
         }
     } else {
-        for (int r = threadIdx.x; r < R; r += kThreads) {
+        for (int r = threadIdx.x; r < R; r += NT) {
             int32_t c = 0;
             for (int tl = 0; tl < P.nt; ++tl) c += (s.mask[tl * rw + (r >> 5)] >> (r & 31)) & 1u;
             s.hr[r] = c;
@@ -288,12 +362,13 @@ __device__ void rank_counts(int k, int R, const Smem &s, const Pairs &P) {
 }
 
 // is_token_in_rank rows of the block (contiguous; 16-byte aligned when R % 16 == 0).
-__device__ void write_rank_rows(int R, uint8_t *__restrict__ in_rank, const Smem &s, const Pairs &P) {
+template <int CH = kChunks, int NT = kThreads>
+__device__ void write_rank_rows(int R, uint8_t *__restrict__ in_rank, const Smem &s, const PairsT<CH> &P) {
     const int rw = mask_words(R);
     uint8_t *row0 = in_rank + P.t0 * R;
     const int nbytes = P.nt * R;
     if ((R & 15) == 0) {
-        for (int q = threadIdx.x * 16; q < nbytes; q += kThreads * 16) {
+        for (int q = threadIdx.x * 16; q < nbytes; q += NT * 16) {
             const int tl = q / R, r0 = q - tl * R;
             const uint32_t bits = (s.mask[tl * rw + (r0 >> 5)] >> (r0 & 31)) & 0xFFFFu;
             uint32_t wv[4];
@@ -302,7 +377,7 @@ __device__ void write_rank_rows(int R, uint8_t *__restrict__ in_rank, const Smem
             *reinterpret_cast<uint4 *>(row0 + q) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
     } else {
-        for (int q = threadIdx.x; q < nbytes; q += kThreads) {
+        for (int q = threadIdx.x; q < nbytes; q += NT) {
             const int tl = q / R, r = q - tl * R;
             row0[q] = (uint8_t)((s.mask[tl * rw + (r >> 5)] >> (r & 31)) & 1u);
         }
@@ -386,9 +461,10 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
 
 // Exclusive scan of v[0..n) in shared memory (n <= kMaxExperts) into out[];
 // returns the total.  All threads of the block must call it.
+template <int NT = kThreads>
 __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, int32_t *warp_sums) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (n + kThreads - 1) / kThreads;   // <= 4
+    const int per = (n + NT - 1) / NT;   // <= 4
     const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
     int32_t local = 0;
     for (int i = i0; i < i1; ++i) local += v[i];
@@ -401,13 +477,13 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int32_t s = lane < kWarps ? warp_sums[lane] : 0;
+        int32_t s = lane < (NT / 32) ? warp_sums[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int32_t u = __shfl_up_sync(0xFFFFFFFFu, s, o);
             if (lane >= o) s += u;
         }
-        if (lane < kWarps) warp_sums[lane] = s;   // inclusive over warps
+        if (lane < (NT / 32)) warp_sums[lane] = s;   // inclusive over warps
     }
     __syncthreads();
     int32_t run = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - local;
@@ -415,23 +491,25 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
         out[i] = run;
         run += v[i];
     }
-    const int32_t total = warp_sums[kWarps - 1];
+    const int32_t total = warp_sums[(NT / 32) - 1];
     __syncthreads();
     return total;
 }
 
 // Bases, the global outputs (block 0) and the rows of the block's pairs.
-template <bool kCoherent, bool kRankKeys>
+// kTotalsGiven: s.total / s.base (copies in earlier blocks) are already set.
+template <bool kCoherent, bool kRankKeys, int CH = kChunks, bool kTotalsGiven = false, int NT = kThreads>
 __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t n, int k, int E, int R,
                                int cap, int64_t recv_rows, int32_t *__restrict__ tokens_per_expert,
                                int32_t *__restrict__ tokens_per_rank, int32_t *__restrict__ expert_offset,
                                int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
                                int32_t *__restrict__ recv_src, uint32_t *status, const Smem &s,
-                               const Pairs &P, int32_t *scan_tmp) {
+                               const PairsT<CH> &P, int32_t *scan_tmp) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nb = gridDim.x, b = blockIdx.x;
-    if (nb == 1) {   // one block: its own counts are the totals
-        for (int e = tid; e < E; e += kThreads) {
+    if constexpr (kTotalsGiven) {
+    } else if (nb == 1) {   // one block: its own counts are the totals
+        for (int e = tid; e < E; e += NT) {
             s.total[e] = s.he[e];
             s.base[e] = 0;
         }
@@ -439,12 +517,12 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
     } else {
         column_sums<kCoherent>(ws_e, nb, E, b, s.total, s.base, s.part);
     }
-    const int32_t m_total = block_exclusive_scan(s.total, s.off, E, scan_tmp);
-    for (int e = tid; e < E; e += kThreads) s.base[e] += cap > 0 ? e * cap : s.off[e];
+    const int32_t m_total = block_exclusive_scan<NT>(s.total, s.off, E, scan_tmp);
+    for (int e = tid; e < E; e += NT) s.base[e] += cap > 0 ? e * cap : s.off[e];
 
     if (b == 0) {
         int32_t mx = 0;
-        for (int e = tid; e < E; e += kThreads) {
+        for (int e = tid; e < E; e += NT) {
             tokens_per_expert[e] = s.total[e];
             expert_offset[e] = s.off[e];
             mx = max(mx, s.total[e]);
@@ -456,35 +534,37 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         __syncthreads();
         if (tid == 0) {
             int32_t m = 0;
-            for (int w = 0; w < kWarps; ++w) m = max(m, scan_tmp[w]);
+            for (int w = 0; w < (NT / 32); ++w) m = max(m, scan_tmp[w]);
             *max_count = m;
         }
         // tokens_per_rank: column sums of the rank table (s.part is free again)
-        if (tokens_per_rank == nullptr) {
-        } else if (nb == 1 && s.hr != nullptr) {
-            for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
-        } else {
-            column_sums<kCoherent>(ws_r, nb, R, 0, s.off, nullptr, s.part);
-            for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.off[r];
+        if constexpr (!kTotalsGiven) {
+            if (tokens_per_rank == nullptr) {
+            } else if (nb == 1 && s.hr != nullptr) {
+                for (int r = tid; r < R; r += NT) tokens_per_rank[r] = s.hr[r];
+            } else {
+                column_sums<kCoherent>(ws_r, nb, R, 0, s.off, nullptr, s.part);
+                for (int r = tid; r < R; r += NT) tokens_per_rank[r] = s.off[r];
+            }
         }
     }
 
-    const int64_t step = (int64_t)nb * kThreads;
+    const int64_t step = (int64_t)nb * NT;
     if (cap > 0) {
         const int64_t rows = (int64_t)E * cap;
-        for (int64_t i = (int64_t)b * kThreads + tid; i < rows; i += step) {
+        for (int64_t i = (int64_t)b * NT + tid; i < rows; i += step) {
             const int e = (int)(i / cap);
             if (i - (int64_t)e * cap >= s.total[e]) recv_src[i] = -1;
         }
     } else {
-        for (int64_t i = m_total + (int64_t)b * kThreads + tid; i < n * k; i += step) recv_src[i] = -1;
+        for (int64_t i = m_total + (int64_t)b * NT + tid; i < n * k; i += step) recv_src[i] = -1;
     }
     __syncthreads();
 
     bool over = false, bad_row = false;
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int p = pair_of(i);
+    for (int i = 0; i < CH; ++i) {
+        const int p = pair_of<CH>(i);
         if (p >= P.np) continue;
         const int32_t e = P.e[i];
         int32_t d = -1;
@@ -503,20 +583,25 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
     if (bad_row) report(status, kErrRange);
 }
 
-// Wait until flags[0..nb) all hold `tag` (acquire), polling one flag per
-// thread at a time, for at most kWaitCycles (~1 s).  Returns true for the
-// whole block when every flag was seen; otherwise reports CGL_ETIMEOUT and
-// returns false for the whole block.  All threads of the block must call it.
+// Wait until flags[0..nb) all hold `tag`, for at most kWaitCycles (~1 s).
+// Warp 0 polls (lane l watches flags l, l + 32, ...) with relaxed loads, so a
+// poll costs one L2 read and no L1 invalidation; once every flag has been seen
+// a gpu-scope fence makes the other blocks' earlier writes visible, and the
+// block barrier hands that on to the whole block.  Returns true for the whole
+// block when every flag was seen; otherwise reports CGL_ETIMEOUT and returns
+// false for the whole block.  All threads of the block must call it.
 __device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint32_t *status) {
     bool timed_out = false;
-    const long long start = clock64();
-    for (int bb = threadIdx.x; bb < nb && !timed_out; bb += kThreads) {
-        while (ld_acquire_u64(flags + bb) != tag) {
-            if (clock64() - start > kWaitCycles) { timed_out = true; break; }
-            __nanosleep(64);
+    if (threadIdx.x < 32) {
+        const long long start = clock64();
+        for (int bb = threadIdx.x; bb < nb && !timed_out; bb += 32) {
+            while (ld_relaxed_u64(flags + bb) != tag) {
+                if (clock64() - start > kWaitCycles) { timed_out = true; break; }
+                __nanosleep(32);
+            }
         }
+        __threadfence();
     }
-    __threadfence();
     if (__syncthreads_or(timed_out)) {
         if (threadIdx.x == 0) report(status, 1u << CGL_ETIMEOUT);
         return false;
@@ -532,8 +617,9 @@ __global__ void __launch_bounds__(kThreads) wait_probe_kernel(const uint64_t *fl
     wait_for_flags(flags, nflags, kTagHigh, status);
 }
 
+template <int NT = kThreads>
 __device__ void zero_words(int32_t *p, int n) {
-    for (int i = threadIdx.x; i < n; i += kThreads) p[i] = 0;
+    for (int i = threadIdx.x; i < n; i += NT) p[i] = 0;
 }
 
 // ------------------------------------------------------------------ kernels
@@ -541,7 +627,7 @@ __device__ void zero_words(int32_t *p, int n) {
 // Kernel arguments: E = number of keys (experts, or ranks in rank mode),
 // E_ids / key_div = valid id range and expert-to-rank divisor for the key
 // transform.  in_rank == nullptr skips the rank sets (rank mode).
-template <bool kRankKeys>
+template <bool kRankKeys, int CH>
 __global__ void __launch_bounds__(kThreads)
 layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
                     int key_div, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
@@ -564,22 +650,22 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const uint64_t g0 = ld_relaxed_u64(gen) & 0xFFFFFFFFull;
     const uint64_t tag = kTagHigh | ((g0 + 1) & 0xFFFFFFFFull);
     zero_words(s.wc, kWarps * E);
-    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
+    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k, CH) * mask_words(R));
     zero_words(s.hr, R);
     __syncthreads();
-    Pairs P;
-    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
-    if (with_ranks) rank_sets(k, E, R, s, P);
+    PairsT<CH> P;
+    const bool bad = load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
+    if (with_ranks) rank_sets<CH>(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
     if (with_ranks) {
-        rank_counts(k, R, s, P);
-        write_rank_rows(R, in_rank, s, P);
+        rank_counts<CH>(k, R, s, P);
+        write_rank_rows<CH>(R, in_rank, s, P);
     }
     __syncthreads();
     if (nb == 1) {   // nothing to exchange
         if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
-        bases_and_rows<true, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+        bases_and_rows<true, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                         tokens_per_rank, expert_offset, max_count, dst_pos, recv_src,
                                         status, s, P, scan_tmp);
         return;
@@ -596,12 +682,13 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     // every block's counts must be visible before the bases
     if (!wait_for_flags(flags, nb, tag, status)) return;
     if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
-    bases_and_rows<true, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+
+    bases_and_rows<true, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                     tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
                                     s, P, scan_tmp);
 }
 
-template <bool kRankKeys>
+template <bool kRankKeys, int CH>
 __global__ void __launch_bounds__(kThreads)
 layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int E_ids, int key_div,
                     int32_t *__restrict__ ws_e, int32_t *__restrict__ ws_r,
@@ -611,17 +698,17 @@ layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const int tid = threadIdx.x;
     const bool with_ranks = in_rank != nullptr;
     zero_words(s.wc, kWarps * E);
-    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
+    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k, CH) * mask_words(R));
     zero_words(s.hr, R);
     __syncthreads();
-    Pairs P;
-    const bool bad = load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
-    if (with_ranks) rank_sets(k, E, R, s, P);
+    PairsT<CH> P;
+    const bool bad = load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
+    if (with_ranks) rank_sets<CH>(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
     if (with_ranks) {
-        rank_counts(k, R, s, P);
-        write_rank_rows(R, in_rank, s, P);
+        rank_counts<CH>(k, R, s, P);
+        write_rank_rows<CH>(R, in_rank, s, P);
     }
     __syncthreads();
     for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)blockIdx.x * E + i] = s.he[i];
@@ -629,7 +716,7 @@ layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
 }
 
-template <bool kRankKeys>
+template <bool kRankKeys, int CH>
 __global__ void __launch_bounds__(kThreads)
 layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
                    int key_div, const int32_t *__restrict__ ws_e, const int32_t *__restrict__ ws_r,
@@ -644,13 +731,13 @@ layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int
     __syncthreads();
     // topk_idx is not written by the counts kernel, which started only after
     // everything before it in the stream had finished: it may be read before the wait
-    Pairs P;
-    load_and_rank<kRankKeys>(idx, n, k, E_ids, key_div, E, blockIdx.x, s, P);
+    PairsT<CH> P;
+    load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
     __syncthreads();
     warp_offsets(E, s);
     griddep_wait();
     __syncthreads();
-    bases_and_rows<false, kRankKeys>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
+    bases_and_rows<false, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                      tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
                                      s, P, scan_tmp);
 }
@@ -680,7 +767,7 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     zero_words(s.hr, R);
     __syncthreads();
     Pairs P;
-    const bool bad = load_and_rank<false>(idx, n, k, E, E / R, E, 0, s, P);
+    const bool bad = load_and_rank<false>(idx, n, k, E, E / R, E, 0, tokens_per_block(k), s, P);
     if (writer) rank_sets(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
@@ -774,18 +861,20 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 // ------------------------------------------------------------------ host side
 
 std::mutex g_mu;
-int g_fused_ctas_per_sm[2][64] = {{0}};   // fused-kernel occupancy at kSmemDefault, per mode and device
+int g_fused_ctas_per_sm[2][3][64] = {{{0}}};   // fused-kernel occupancy at kSmemDefault, per mode, CH, device
+
+__host__ __device__ constexpr int ch_slot(int ch) { return ch == 1 ? 0 : (ch == 2 ? 1 : 2); }
 
 // Largest grid of the fused kernel that is certain to be co-resident; 0 if none.
-template <bool kRankKeys>
+template <bool kRankKeys, int CH>
 int fused_capacity() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(g_mu);
-    int &slot = g_fused_ctas_per_sm[kRankKeys ? 1 : 0][dev];
+    int &slot = g_fused_ctas_per_sm[kRankKeys ? 1 : 0][ch_slot(CH)][dev];
     if (slot == 0) {
         int v = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, layout_fused_kernel<kRankKeys>, kThreads,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, layout_fused_kernel<kRankKeys, CH>, kThreads,
                                                           kSmemDefault) != cudaSuccess)
             return 0;
         slot = v > 0 ? v : -1;
@@ -796,8 +885,12 @@ int fused_capacity() {
 template <bool kRankKeys>
 bool fused_fits(int64_t n, int k, int nkeys, int R) {
     const WsLayout w = ws_layout(n, k, nkeys, R);
-    return smem_words(0, k, nkeys, R) * sizeof(int32_t) <= kSmemDefault &&
-           w.blocks <= fused_capacity<kRankKeys>();
+    if (smem_words(0, k, nkeys, R) * sizeof(int32_t) > kSmemDefault) return false;
+    switch (layout_chunks(n, k)) {
+        case 1: return w.blocks <= fused_capacity<kRankKeys, 1>();
+        case 2: return w.blocks <= fused_capacity<kRankKeys, 2>();
+        default: return w.blocks <= fused_capacity<kRankKeys, 4>();
+    }
 }
 
 }  // namespace
@@ -810,11 +903,11 @@ bool layout_needs_smem_optin(int E, int R, int k) {
 
 bool layout_fused_fits(int64_t n, int k, int E, int R) { return fused_fits<false>(n, k, E, R); }
 
-template <bool kRankKeys>
-cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
-                              int32_t *tokens_per_key, int32_t *tokens_per_rank, uint8_t *in_rank,
-                              int32_t *key_offset, int32_t *max_count, int32_t *dst_pos,
-                              int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+template <bool kRankKeys, int CH>
+cgl_status launch_layout_ch(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
+                            int32_t *tokens_per_key, int32_t *tokens_per_rank, uint8_t *in_rank,
+                            int32_t *key_offset, int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
+                            void *ws, uint32_t *status, cudaStream_t stream) {
     const int E = kRankKeys ? R : E_ids;        // number of keys
     const int key_div = E_ids / R;
     const WsLayout w = ws_layout(n, k, E, R);
@@ -835,7 +928,7 @@ cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, i
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const cudaError_t err = cudaLaunchKernelEx(
-            &cfg, layout_fused_kernel<kRankKeys>, idx, n, k, E, R, cap, E_ids, key_div, flags, ws_e, ws_r,
+            &cfg, layout_fused_kernel<kRankKeys, CH>, idx, n, k, E, R, cap, E_ids, key_div, flags, ws_e, ws_r,
             tokens_per_key, tokens_per_rank, in_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
             status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
@@ -843,19 +936,40 @@ cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, i
 
     const size_t smem1 = smem_words(1, k, E, R) * sizeof(int32_t);
     const size_t smem2 = smem_words(2, k, E, R) * sizeof(int32_t);
-    if (smem1 > kSmemDefault && !ensure_smem_attr((const void *)layout_count_kernel<kRankKeys>, smem1))
+    if (smem1 > kSmemDefault && !ensure_smem_attr((const void *)layout_count_kernel<kRankKeys, CH>, smem1))
         return CGL_ECUDA;
-    if (smem2 > kSmemDefault && !ensure_smem_attr((const void *)layout_rows_kernel<kRankKeys>, smem2))
+    if (smem2 > kSmemDefault && !ensure_smem_attr((const void *)layout_rows_kernel<kRankKeys, CH>, smem2))
         return CGL_ECUDA;
-    layout_count_kernel<kRankKeys><<<(unsigned)w.blocks, kThreads, smem1, stream>>>(
+    layout_count_kernel<kRankKeys, CH><<<(unsigned)w.blocks, kThreads, smem1, stream>>>(
         idx, n, k, E, R, E_ids, key_div, ws_e, ws_r, in_rank, status);
     if (cudaGetLastError() != cudaSuccess) return CGL_ECUDA;
-    const cudaError_t err = launch_pdl(layout_rows_kernel<kRankKeys>, dim3((unsigned)w.blocks), dim3(kThreads),
+    const cudaError_t err = launch_pdl(layout_rows_kernel<kRankKeys, CH>, dim3((unsigned)w.blocks), dim3(kThreads),
                                        smem2, stream, idx, n, k, E, R, cap, E_ids, key_div,
                                        (const int32_t *)ws_e, (const int32_t *)ws_r, tokens_per_key,
                                        tokens_per_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
                                        status);
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+}
+
+template <bool kRankKeys>
+cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
+                              int32_t *tokens_per_key, int32_t *tokens_per_rank, uint8_t *in_rank,
+                              int32_t *key_offset, int32_t *max_count, int32_t *dst_pos,
+                              int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+    switch (layout_chunks(n, k)) {
+        case 1:
+            return launch_layout_ch<kRankKeys, 1>(idx, n, k, E_ids, R, cap, tokens_per_key, tokens_per_rank,
+                                                  in_rank, key_offset, max_count, dst_pos, recv_src, ws, status,
+                                                  stream);
+        case 2:
+            return launch_layout_ch<kRankKeys, 2>(idx, n, k, E_ids, R, cap, tokens_per_key, tokens_per_rank,
+                                                  in_rank, key_offset, max_count, dst_pos, recv_src, ws, status,
+                                                  stream);
+        default:
+            return launch_layout_ch<kRankKeys, 4>(idx, n, k, E_ids, R, cap, tokens_per_key, tokens_per_rank,
+                                                  in_rank, key_offset, max_count, dst_pos, recv_src, ws, status,
+                                                  stream);
+    }
 }
 
 cgl_status launch_layout(const int32_t *idx, int64_t n, int k, int E, int R, int cap,

@@ -54,6 +54,18 @@ def test_layout_random_ragged(oracle_mod, seed):
     run_both(oracle_mod, idx, E, R, 0)
 
 
+@pytest.mark.parametrize("n,k", [(4096, 8), (4097, 8), (8192, 8), (8193, 8), (5462, 6), (43, 6)])
+def test_layout_block_size_boundaries(oracle_mod, n, k):
+    """Token counts on both sides of a change of block size (32 -> 64 -> 128
+    tokens per block at k = 8 once the grid would pass 128 blocks), padded too."""
+    rng = np.random.default_rng(n * 31 + k)
+    E, R = 256, 64
+    idx = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    idx[rng.random((n, k)) < 0.03] = -1
+    lay, _ = run_both(oracle_mod, idx, E, R, 0)
+    run_both(oracle_mod, idx, E, R, max(1, int(lay.max_count.item()) - 3))   # a few copies over capacity
+
+
 def test_layout_duplicates_bad_ids_and_overflow(oracle_mod):
     rng = np.random.default_rng(42)
     n, k, E, R = 700, 8, 16, 4

@@ -87,8 +87,8 @@ def test_noalloc_refuses_sizes_past_its_scratch():
     fake = 1 << 16   # never dereferenced: the size check comes first
     f = _fn()
     args = [fake] * 7
-    # 60000 tokens at E=256, R=64 need more than the 256 KiB scratch array
-    assert cgl.layout_workspace_bytes(60000, 8, 256, 64) > 256 * 1024
+    # 60000 tokens at E=256, R=64 need more than the 512 KiB scratch array
+    assert cgl.layout_workspace_bytes(60000, 8, 256, 64) > 512 * 1024
     assert f(fake, 60000, 8, 256, 64, None, *args, None, None) == cgl.EINVAL
     # E=1024 with k=8 would need more than 48 KiB of shared memory per block
     assert f(fake, 100, 8, 1024, 64, None, *args, None, None) == cgl.EINVAL
