@@ -250,11 +250,16 @@ __device__ __forceinline__ void key_and_rank(const int32_t *__restrict__ idx, in
             }
         }
     }
+    // the matches of all chunks first (independent, so their latencies overlap),
+    // then the chain through the warp's counters
+    unsigned grp[CH];
+#pragma unroll
+    for (int i = 0; i < CH; ++i) grp[i] = __match_any_sync(0xFFFFFFFFu, P.e[i]);
     int32_t *wc = s.wc + warp * nkeys;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
         const int32_t e = P.e[i];
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        const unsigned peers = grp[i];
         const int32_t before = e >= 0 ? wc[e] : 0;
         __syncwarp();
         if (e >= 0 && (peers & lower) == 0) wc[e] = before + __popc(peers);
@@ -344,6 +349,7 @@ __device__ void rank_counts(int k, int R, const Smem &s, const PairsT<CH> &P) {
                 if (rw > 1) m |= (uint64_t)s.mask[tl * rw + 1] << 32;
             }
             int32_t c0 = 0, c1 = 0;
+#pragma unroll 4
             for (int r = r0; r < r1; ++r) {
                 const int c = __popc(__ballot_sync(0xFFFFFFFFu, (m >> r) & 1ull));
                 if (r == lane) c0 = c;
@@ -507,6 +513,21 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
                                const PairsT<CH> &P, int32_t *scan_tmp) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nb = gridDim.x, b = blockIdx.x;
+    // tokens_per_rank from the table (unless this is the only block and it has
+    // its own counts): rank column r is summed by warp (r / nb) % 8 of block
+    // r % nb.  The loads of a warp's first column are issued before the expert
+    // column sums and added after them, so both wait out the same round trip.
+    const bool rank_sums = !kTotalsGiven && tokens_per_rank != nullptr && !(nb == 1 && s.hr != nullptr);
+    const int rcol = b + warp * nb;
+    int32_t rv[4] = {0, 0, 0, 0};
+    if (rank_sums && rcol < R) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = lane + 32 * q;
+            if (i < nb) rv[q] = ld_col1<kCoherent>(ws_r + (int64_t)i * R + rcol);
+        }
+        for (int i = lane + 128; i < nb; i += 32) rv[0] += ld_col1<kCoherent>(ws_r + (int64_t)i * R + rcol);
+    }
     if constexpr (kTotalsGiven) {
     } else if (nb == 1) {   // one block: its own counts are the totals
         for (int e = tid; e < E; e += NT) {
@@ -516,6 +537,19 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         __syncthreads();
     } else {
         column_sums<kCoherent>(ws_e, nb, E, b, s.total, s.base, s.part);
+    }
+    if (rank_sums) {
+        for (int r = rcol; r < R; r += nb * (NT / 32)) {   // warp-uniform
+            int32_t v = 0;
+            if (r == rcol) {
+                v = rv[0] + rv[1] + rv[2] + rv[3];
+            } else {
+                for (int i = lane; i < nb; i += 32) v += ld_col1<kCoherent>(ws_r + (int64_t)i * R + r);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            if (lane == 0) tokens_per_rank[r] = v;
+        }
     }
     const int32_t m_total = block_exclusive_scan<NT>(s.total, s.off, E, scan_tmp);
     for (int e = tid; e < E; e += NT) s.base[e] += cap > 0 ? e * cap : s.off[e];
@@ -537,15 +571,10 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
             for (int w = 0; w < (NT / 32); ++w) m = max(m, scan_tmp[w]);
             *max_count = m;
         }
-        // tokens_per_rank: column sums of the rank table (s.part is free again)
+        // tokens_per_rank of a single block: its own distinct-token counts
         if constexpr (!kTotalsGiven) {
-            if (tokens_per_rank == nullptr) {
-            } else if (nb == 1 && s.hr != nullptr) {
+            if (tokens_per_rank != nullptr && nb == 1 && s.hr != nullptr)
                 for (int r = tid; r < R; r += NT) tokens_per_rank[r] = s.hr[r];
-            } else {
-                column_sums<kCoherent>(ws_r, nb, R, 0, s.off, nullptr, s.part);
-                for (int r = tid; r < R; r += NT) tokens_per_rank[r] = s.off[r];
-            }
         }
     }
 
@@ -584,21 +613,22 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
 }
 
 // Wait until flags[0..nb) all hold `tag`, for at most kWaitCycles (~1 s).
-// Warp 0 polls (lane l watches flags l, l + 32, ...) with relaxed loads, so a
-// poll costs one L2 read and no L1 invalidation; once every flag has been seen
-// a gpu-scope fence makes the other blocks' earlier writes visible, and the
-// block barrier hands that on to the whole block.  Returns true for the whole
+// Warp 0 polls: each round, lane l reads flags l, l + 32, ... with relaxed
+// loads (one L2 read each, no L1 invalidation, all in flight together) until
+// every lane has seen its flags; then a gpu-scope fence makes the other
+// blocks' earlier writes visible, and the block barrier hands that on to the
+// whole block.  Returns true for the whole
 // block when every flag was seen; otherwise reports CGL_ETIMEOUT and returns
 // false for the whole block.  All threads of the block must call it.
 __device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint32_t *status) {
     bool timed_out = false;
     if (threadIdx.x < 32) {
         const long long start = clock64();
-        for (int bb = threadIdx.x; bb < nb && !timed_out; bb += 32) {
-            while (ld_relaxed_u64(flags + bb) != tag) {
-                if (clock64() - start > kWaitCycles) { timed_out = true; break; }
-                __nanosleep(32);
-            }
+        for (;;) {
+            bool seen = true;
+            for (int bb = threadIdx.x; bb < nb; bb += 32) seen &= ld_relaxed_u64(flags + bb) == tag;
+            if (__all_sync(0xFFFFFFFFu, seen)) break;
+            if (__any_sync(0xFFFFFFFFu, clock64() - start > kWaitCycles)) { timed_out = true; break; }
         }
         __threadfence();
     }
@@ -649,21 +679,20 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     flags += 1;
     const uint64_t g0 = ld_relaxed_u64(gen) & 0xFFFFFFFFull;
     const uint64_t tag = kTagHigh | ((g0 + 1) & 0xFFFFFFFFull);
+    PairsT<CH> P;
+    const bool bad = load_pairs<CH>(idx, n, k, E_ids, b, tokens_per_block(k, CH), P);   // in flight while zeroing
     zero_words(s.wc, kWarps * E);
     zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k, CH) * mask_words(R));
     zero_words(s.hr, R);
     __syncthreads();
-    PairsT<CH> P;
-    const bool bad = load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
+    key_and_rank<kRankKeys, CH>(idx, k, E_ids, key_div, E, s, P);
     if (with_ranks) rank_sets<CH>(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
-    if (with_ranks) {
-        rank_counts<CH>(k, R, s, P);
-        write_rank_rows<CH>(R, in_rank, s, P);
-    }
+    if (with_ranks) rank_counts<CH>(k, R, s, P);
     __syncthreads();
     if (nb == 1) {   // nothing to exchange
+        if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
         if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
         bases_and_rows<true, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
                                         tokens_per_rank, expert_offset, max_count, dst_pos, recv_src,
@@ -678,6 +707,9 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         st_release_u64(flags + b, tag);
         if (any_bad) report(status, kErrRange);
     }
+    // no other block reads these rows: written after the flag, so the fence above
+    // does not wait for them
+    if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
 
     // every block's counts must be visible before the bases
     if (!wait_for_flags(flags, nb, tag, status)) return;
