@@ -44,7 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {
     "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
     "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
-    "layout": {"bytes": 210176, "src_sha": "55a9ef26e30253f8"},
+    "layout": {"bytes": 206080, "src_sha": "2315501c74f4a785"},
 }
 
 
