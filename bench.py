@@ -181,7 +181,7 @@ class GpuStep:
     """Device buffers for one workload and the launch sequence of one step."""
 
     def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False, full_backward: bool = False,
-                 fused_decode: bool = False):
+                 fused_decode: bool = False, split_layout: bool = False):
         import torch
 
         import combine_get_layout_02_b200 as cgl
@@ -190,6 +190,9 @@ class GpuStep:
         self.dedup = dedup
         self.full_backward = full_backward and wl.with_grad and not dedup
         self.fused_decode = fused_decode and wl.fp8 and not dedup
+        # FP8 steps call cgl_layout_dispatch_fp8 (one cooperative kernel when it
+        # applies, else the layout and dispatch kernels) unless asked to split
+        self.layout_dispatch = wl.fp8 and not dedup and not self.fused_decode and not split_layout
         inp = W.make_inputs(wl, seed)
         n, h, k = wl.num_tokens, wl.hidden, wl.topk
         self.host = inp
@@ -207,7 +210,8 @@ class GpuStep:
         self.grad = bf16(inp.grad).to(device) if inp.grad is not None else None
         self.status = cgl.new_status(device)
         E, R = wl.num_experts, wl.num_ranks
-        self.ws = torch.empty(cgl.layout_workspace_bytes(n, k, E, R), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(max(cgl.layout_workspace_bytes(n, k, E, R),
+                                  cgl.layout_dispatch_workspace_bytes(n, k, E, R)), dtype=torch.uint8, device=device)
         self.cap = 0
         if wl.padded:   # padded receive buffers: size them from a first compact call (host reads max)
             lay = cgl.get_layout(self.idx, E, R, 0, workspace=self.ws, status=self.status)
@@ -259,6 +263,10 @@ class GpuStep:
             ph = [("layout+dispatch_fp8", 1, b["layout"] + b["dispatch_fp8"]),
                   ("combine", 1, b["combine"])]
             return ph
+        if self.layout_dispatch:
+            nk = self.cgl.layout_dispatch_kernel_count(wl.num_tokens, wl.topk, wl.num_experts, wl.num_ranks,
+                                                       wl.hidden)
+            return [("layout+dispatch_fp8", nk, b["layout"] + b["dispatch_fp8"]), ("combine", 1, b["combine"])]
         if self.dedup:   # rank keys: the layout of an E = R problem
             nl = self.cgl.layout_kernel_count(wl.num_tokens, wl.topk, wl.num_ranks, wl.num_ranks)
         else:
@@ -289,6 +297,13 @@ class GpuStep:
         if self.fused_decode:
             cgl.decode_dispatch_fp8(self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x,
                                     recv_scale=self.recv_scale, status=self.status)
+            rec()
+            cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
+            rec()
+            return
+        if self.layout_dispatch:
+            cgl.layout_dispatch_fp8(self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x,
+                                    recv_scale=self.recv_scale, workspace=self.ws, status=self.status)
             rec()
             cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
             rec()
@@ -552,7 +567,7 @@ def run_ours(args):
 
         wl = dataclasses.replace(wl, num_tokens=args.num_tokens)
     step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup, full_backward=args.full_backward,
-                   fused_decode=args.fused_decode)
+                   fused_decode=args.fused_decode, split_layout=args.split_layout)
     phases = step.kernels()
 
     graph = None if args.no_graph else capture_step(step)
@@ -680,6 +695,8 @@ def main(argv=None):
                     help="bf16 workload: weighted combine backward with grad_w instead of the plain re-dispatch")
     ap.add_argument("--fused-decode", action="store_true",
                     help="layout and FP8 dispatch in one launch (batches of at most 1024 token-slot pairs)")
+    ap.add_argument("--split-layout", action="store_true",
+                    help="FP8: cgl_get_layout and cgl_dispatch_fp8 as two calls instead of cgl_layout_dispatch_fp8")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -84,6 +84,13 @@ def lib():
         L.cgl_combine.restype = I
         L.cgl_decode_dispatch_fp8.argtypes = [P, I64, I, I, I, OP, P, I, P, P, P, P, P, P, P, P, P, P, P]
         L.cgl_decode_dispatch_fp8.restype = I
+        L.cgl_layout_dispatch_workspace_bytes.argtypes = [I64, I, I, I]
+        L.cgl_layout_dispatch_workspace_bytes.restype = C.c_size_t
+        L.cgl_layout_dispatch_kernel_count.argtypes = [I64, I, I, I, I, OP]
+        L.cgl_layout_dispatch_kernel_count.restype = I
+        L.cgl_layout_dispatch_fp8.argtypes = [P, I64, I, I, I, OP, P, I, P, P, P, P, P, P, P, P, P, P,
+                                              C.c_size_t, P, P]
+        L.cgl_layout_dispatch_fp8.restype = I
         L.cgl_combine_backward.argtypes = [P, P, I64, P, P, I64, I, I, P, P, OP, P, P]
         L.cgl_combine_backward.restype = I
         _lib = L
@@ -349,4 +356,57 @@ def decode_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: in
         _ptr(out.tokens_per_rank), _ptr(out.is_token_in_rank), _ptr(out.expert_offset), _ptr(out.max_count),
         _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(recv_x), _ptr(recv_scale), _ptr(status), _stream(stream))
     _check(code, "cgl_decode_dispatch_fp8")
+    return out, recv_x, recv_scale
+
+
+def layout_dispatch_workspace_bytes(num_tokens: int, num_topk: int, num_experts: int, num_ranks: int) -> int:
+    return int(lib().cgl_layout_dispatch_workspace_bytes(num_tokens, num_topk, num_experts, num_ranks))
+
+
+def layout_dispatch_kernel_count(num_tokens: int, num_topk: int, num_experts: int, num_ranks: int,
+                                 hidden: int, num_sms: int = 0) -> int:
+    return int(lib().cgl_layout_dispatch_kernel_count(num_tokens, num_topk, num_experts, num_ranks, hidden,
+                                                      _opts(num_sms, 0)))
+
+
+def layout_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: int, num_ranks: int,
+                        capacity: int = 0, *, out: Optional[Layout] = None,
+                        recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                        num_sms: int = 0, stream=None):
+    """Layout + FP8 dispatch of any batch in one call (cgl_layout_dispatch_fp8).
+
+    Returns (Layout, recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128])."""
+    idx = _dev(topk_idx, "topk_idx", torch.int32, 2)
+    x = _dev(x, "x", torch.bfloat16, 2)
+    n, k = idx.shape
+    h = x.shape[1]
+    E, R = int(num_experts), int(num_ranks)
+    dev = idx.device
+    rows = E * capacity if capacity > 0 else n * k
+    ws_bytes = layout_dispatch_workspace_bytes(n, k, E, R)
+    if ws_bytes == 0:
+        raise CglError(EINVAL, "layout_dispatch_fp8", "invalid sizes")
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = Layout(
+            torch.empty(E, dtype=torch.int32, device=dev),
+            torch.empty(R, dtype=torch.int32, device=dev),
+            torch.empty((n, R), dtype=torch.uint8, device=dev),
+            torch.empty(E + 1, dtype=torch.int32, device=dev),
+            torch.empty(1, dtype=torch.int32, device=dev),
+            torch.empty((n, k), dtype=torch.int32, device=dev),
+            torch.empty(rows, dtype=torch.int32, device=dev),
+            rows, int(capacity))
+    if recv_x is None:
+        recv_x = torch.empty((rows, h), dtype=torch.uint8, device=dev)
+    if recv_scale is None:
+        recv_scale = torch.empty((rows, h // 128), dtype=torch.float32, device=dev)
+    code = lib().cgl_layout_dispatch_fp8(
+        _ptr(idx), n, k, E, R, _opts(num_sms, capacity), _ptr(x), h, _ptr(out.tokens_per_expert),
+        _ptr(out.tokens_per_rank), _ptr(out.is_token_in_rank), _ptr(out.expert_offset), _ptr(out.max_count),
+        _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(recv_x), _ptr(recv_scale), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(code, "cgl_layout_dispatch_fp8")
     return out, recv_x, recv_scale

@@ -286,6 +286,44 @@ cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
                                       recv_scale, opt_sms(opts), status_dev, static_cast<cudaStream_t>(stream));
 }
 
+size_t cgl_layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
+    if (!layout_sizes_ok(n, k, E, R)) return 0;
+    return layout_dispatch_workspace_bytes(n, k, E, R);
+}
+
+int cgl_layout_dispatch_kernel_count(int64_t n, int k, int E, int R, int h, const cgl_opts *opts) {
+    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0 || opt_sms(opts) < 0) return -1;
+    if (layout_dispatch_fused_fits(n, k, E, R, h, opt_sms(opts))) return 1;
+    return (layout_fused_fits(n, k, E, R) ? 1 : 2) + 1;
+}
+
+cgl_status cgl_layout_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, int E, int R,
+                                   const cgl_opts *opts, const uint16_t *x, int h,
+                                   int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                                   uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
+                                   int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x, float *recv_scale,
+                                   void *workspace, size_t workspace_bytes, uint32_t *status_dev,
+                                   void *stream) {
+    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0) return CGL_EINVAL;
+    const int cap = opt_cap(opts);
+    if (cap < 0 || (int64_t)E * cap >= ((int64_t)1 << 31) || opt_sms(opts) < 0) return CGL_EINVAL;
+    const int64_t rows = cap > 0 ? (int64_t)E * cap : n * k;
+    if (!tokens_per_expert || !tokens_per_rank || !expert_offset || !max_count || !workspace)
+        return CGL_EINVAL;
+    if (n > 0 && (!topk_idx || !x || !dst_pos || !is_token_in_rank)) return CGL_EINVAL;
+    if (rows > 0 && (!recv_src || !recv_x || !recv_scale)) return CGL_EINVAL;
+    if (workspace_bytes < layout_dispatch_workspace_bytes(n, k, E, R)) return CGL_EINVAL;
+    if (!aligned(topk_idx, 4) || !aligned(x, 16) || !aligned(tokens_per_expert, 4) ||
+        !aligned(tokens_per_rank, 4) || !aligned(is_token_in_rank, 16) || !aligned(expert_offset, 4) ||
+        !aligned(max_count, 4) || !aligned(dst_pos, 4) || !aligned(recv_src, 4) ||
+        !aligned(recv_x, 16) || !aligned(recv_scale, 4) || !aligned(status_dev, 4) || !aligned(workspace, 16))
+        return CGL_EALIGN;
+    return launch_layout_dispatch_fp8(topk_idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank,
+                                      is_token_in_rank, expert_offset, max_count, dst_pos, recv_src, recv_x,
+                                      recv_scale, workspace, opt_sms(opts), status_dev,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 cgl_status cgl_selftest_bounded_wait(const uint64_t *flags, int nflags, uint32_t *status_dev,
                                      void *stream) {
     if (!flags || !status_dev || nflags < 1 || nflags > 4096) return CGL_EINVAL;

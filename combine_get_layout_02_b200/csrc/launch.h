@@ -88,6 +88,17 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       uint8_t *recv_x, float *recv_scale, int num_sms, uint32_t *status,
                                       cudaStream_t stream);
 
+// Fused layout + FP8 dispatch (one cooperative launch when it applies, else
+// the layout and the dispatch kernels in turn).
+size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R);
+bool layout_dispatch_fused_fits(int64_t n, int k, int E, int R, int h, int num_sms);
+cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                                      const uint16_t *x, int h, int32_t *tokens_per_expert,
+                                      int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
+                                      int32_t *max_count, int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
+                                      float *recv_scale, void *ws, int num_sms, uint32_t *status,
+                                      cudaStream_t stream);
+
 cgl_status launch_combine_backward(const uint16_t *g, const uint16_t *y, int64_t recv_rows,
                                    const int32_t *dst_pos, const float *w, int64_t n, int h, int k,
                                    uint16_t *grad_y, float *grad_w, int num_sms, uint32_t *status,

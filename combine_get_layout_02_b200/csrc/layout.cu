@@ -49,9 +49,9 @@
 // every flag shows that tag; one warp polls with relaxed loads and a single
 // fence follows (an acquire load per poll would invalidate L1 every time).
 // One exchange round only: on this part each dependent round trip through L2
-// costs about a microsecond, more than the column sums it would save.  The tag is a generation counter kept in the
-// workspace (+1 per launch), so it changes on every launch, replays of a
-// captured graph included.  Otherwise two kernels run (counts, then bases +
+// costs about a microsecond, more than the column sums it would save.  The
+// tag is a generation counter kept in the workspace (+1 per launch), so it
+// changes on every launch, replays of a captured graph included.  Otherwise two kernels run (counts, then bases +
 // rows), the second with programmatic dependent launch; it recomputes the
 // cheap in-warp ranks.
 #include <mutex>
@@ -104,14 +104,18 @@ struct WsLayout {
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-WsLayout ws_layout(int64_t n, int k, int E, int R) {
+WsLayout ws_layout_blocks(int64_t blocks, int E, int R) {
     WsLayout w;
-    const int T = tokens_per_block(k, layout_chunks(n, k));
-    w.blocks = n > 0 ? (n + T - 1) / T : 1;
+    w.blocks = blocks;
     w.e_off = align256((size_t)(w.blocks + 1) * sizeof(uint64_t));
     w.r_off = w.e_off + align256((size_t)w.blocks * (size_t)E * sizeof(int32_t));
     w.bytes = w.r_off + (size_t)w.blocks * (size_t)R * sizeof(int32_t);
     return w;
+}
+
+WsLayout ws_layout(int64_t n, int k, int E, int R) {
+    const int T = tokens_per_block(k, layout_chunks(n, k));
+    return ws_layout_blocks(n > 0 ? (n + T - 1) / T : 1, E, R);
 }
 
 __device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
@@ -128,6 +132,19 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
 // Flags hold this constant in their high half; counts (non-negative int32) never do.
 constexpr uint64_t kTagHigh = 0x9E3779B9ull << 32;
 
+
+// Barrier of the 256 layout threads (warps 0-7, hardware barrier 1).  In the
+// 256-thread layout kernels that is the whole block; the fused layout +
+// dispatch kernel runs other warps beside them, which never take part.
+__device__ __forceinline__ void lsync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool lsync_or(bool v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, 1, 256, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((int)v) : "memory");
+    return r != 0;
+}
 
 // q = e / d for 0 <= e < 1024 and 1 <= d <= 1024 as (e * m) >> 20 with
 // m = ceil(2^20 / d): exact on that range because e * (m * d - 2^20) < 2^20.
@@ -405,7 +422,7 @@ __device__ __forceinline__ int32_t ld_col1(const int32_t *p) {
 // row needs fewer loads than there are threads, G thread groups split the
 // rows and their partial sums meet in `part`.  kCoherent: the table was
 // written by other blocks of the running grid (read through L2 only).
-template <bool kCoherent>
+template <bool kCoherent, int U = kColUnroll>
 __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32_t *out_tot,
                             int32_t *out_pre, int32_t *part) {
     const int tid = threadIdx.x;
@@ -420,10 +437,10 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
     if (g < G) {
         for (int q = q0; q < nq; q += qstep) {
             int32_t tot[4] = {0, 0, 0, 0}, pre[4] = {0, 0, 0, 0};
-            for (int r0 = g; r0 < nb; r0 += G * kColUnroll) {
-                int4 v[kColUnroll];
+            for (int r0 = g; r0 < nb; r0 += G * U) {
+                int4 v[U];
 #pragma unroll
-                for (int u = 0; u < kColUnroll; ++u) {
+                for (int u = 0; u < U; ++u) {
                     const int r = r0 + u * G;
                     const int32_t *a = t + (int64_t)r * ncols + q * width;
                     if (r >= nb) v[u] = make_int4(0, 0, 0, 0);
@@ -431,7 +448,7 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
                     else v[u] = make_int4(ld_col1<kCoherent>(a), 0, 0, 0);
                 }
 #pragma unroll
-                for (int u = 0; u < kColUnroll; ++u) {
+                for (int u = 0; u < U; ++u) {
                     const int32_t below = r0 + u * G < upto ? 1 : 0;
                     tot[0] += v[u].x; tot[1] += v[u].y; tot[2] += v[u].z; tot[3] += v[u].w;
                     pre[0] += below * v[u].x; pre[1] += below * v[u].y;
@@ -451,7 +468,7 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
         }
     }
     if (G > 1) {
-        __syncthreads();
+        lsync();
         for (int col = tid; col < ncols; col += kThreads) {
             int32_t a = 0, b = 0;
             for (int gg = 0; gg < G; ++gg) {
@@ -462,7 +479,7 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
             if (out_pre) out_pre[col] = b;
         }
     }
-    __syncthreads();
+    lsync();
 }
 
 // Exclusive scan of v[0..n) in shared memory (n <= kMaxExperts) into out[];
@@ -481,7 +498,7 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
         if (lane >= o) incl += u;
     }
     if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
+    lsync();
     if (warp == 0) {
         int32_t s = lane < (NT / 32) ? warp_sums[lane] : 0;
 #pragma unroll
@@ -491,26 +508,27 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
         }
         if (lane < (NT / 32)) warp_sums[lane] = s;   // inclusive over warps
     }
-    __syncthreads();
+    lsync();
     int32_t run = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - local;
     for (int i = i0; i < i1; ++i) {
         out[i] = run;
         run += v[i];
     }
     const int32_t total = warp_sums[(NT / 32) - 1];
-    __syncthreads();
+    lsync();
     return total;
 }
 
 // Bases, the global outputs (block 0) and the rows of the block's pairs.
 // kTotalsGiven: s.total / s.base (copies in earlier blocks) are already set.
-template <bool kCoherent, bool kRankKeys, int CH = kChunks, bool kTotalsGiven = false, int NT = kThreads>
+template <bool kCoherent, bool kRankKeys, int CH = kChunks, bool kTotalsGiven = false, int NT = kThreads,
+          int U = kColUnroll>
 __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t n, int k, int E, int R,
                                int cap, int64_t recv_rows, int32_t *__restrict__ tokens_per_expert,
                                int32_t *__restrict__ tokens_per_rank, int32_t *__restrict__ expert_offset,
                                int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
                                int32_t *__restrict__ recv_src, uint32_t *status, const Smem &s,
-                               const PairsT<CH> &P, int32_t *scan_tmp) {
+                               const PairsT<CH> &P, int32_t *scan_tmp, int32_t *s_dst = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nb = gridDim.x, b = blockIdx.x;
     // tokens_per_rank from the table (unless this is the only block and it has
@@ -534,9 +552,9 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
             s.total[e] = s.he[e];
             s.base[e] = 0;
         }
-        __syncthreads();
+        lsync();
     } else {
-        column_sums<kCoherent>(ws_e, nb, E, b, s.total, s.base, s.part);
+        column_sums<kCoherent, U>(ws_e, nb, E, b, s.total, s.base, s.part);
     }
     if (rank_sums) {
         for (int r = rcol; r < R; r += nb * (NT / 32)) {   // warp-uniform
@@ -565,7 +583,7 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
         if (lane == 0) scan_tmp[warp] = mx;
-        __syncthreads();
+        lsync();
         if (tid == 0) {
             int32_t m = 0;
             for (int w = 0; w < (NT / 32); ++w) m = max(m, scan_tmp[w]);
@@ -588,7 +606,7 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
     } else {
         for (int64_t i = m_total + (int64_t)b * NT + tid; i < n * k; i += step) recv_src[i] = -1;
     }
-    __syncthreads();
+    lsync();
 
     bool over = false, bad_row = false;
 #pragma unroll
@@ -605,6 +623,7 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         }
         const int64_t q = P.t0 * k + p;
         dst_pos[q] = d;
+        if (s_dst) s_dst[p] = d;
         // expert mode: the row's source slot t*k + j; rank mode: its source token t
         if (d >= 0) recv_src[d] = kRankKeys ? (int32_t)(P.t0 + p / k) : (int32_t)q;
     }
@@ -632,7 +651,7 @@ __device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint
         }
         __threadfence();
     }
-    if (__syncthreads_or(timed_out)) {
+    if (lsync_or(timed_out)) {
         if (threadIdx.x == 0) report(status, 1u << CGL_ETIMEOUT);
         return false;
     }
@@ -654,20 +673,21 @@ __device__ void zero_words(int32_t *p, int n) {
 
 // ------------------------------------------------------------------ kernels
 
-// Kernel arguments: E = number of keys (experts, or ranks in rank mode),
-// E_ids / key_div = valid id range and expert-to-rank divisor for the key
-// transform.  in_rank == nullptr skips the rank sets (rank mode).
-template <bool kRankKeys, int CH>
-__global__ void __launch_bounds__(kThreads)
-layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
-                    int key_div, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
-                    int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
-                    uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
-                    int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
-                    int32_t *__restrict__ recv_src, int64_t recv_rows, uint32_t *status) {
-    extern __shared__ __align__(16) int32_t smem_fused[];
-    __shared__ int32_t scan_tmp[32];
-    const Smem s = carve(0, smem_fused, k, E, R);
+// One layout block's whole part of the one-launch layout, run by the 256
+// threads of warps 0-7 (every barrier in it is lsync): block b = blockIdx.x of
+// gridDim.x owns tokens [b T, b T + T).  E = number of keys (experts, or ranks
+// in rank mode), E_ids / key_div = valid id range and expert-to-rank divisor
+// for the key transform; in_rank == nullptr skips the rank sets (rank mode).
+// s_dst (optional, shared memory, T k words) also receives the block's rows.
+// Returns false (the whole group of 256) when the inter-block wait timed out.
+template <bool kRankKeys, int CH, int U = kColUnroll>
+__device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
+                             int key_div, int T, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                             int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
+                             uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
+                             int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
+                             int32_t *__restrict__ recv_src, int64_t recv_rows, uint32_t *status,
+                             const Smem &s, int32_t *scan_tmp, int32_t *s_dst) {
     const int tid = threadIdx.x;
     const int nb = gridDim.x, b = blockIdx.x;
     const bool with_ranks = in_rank != nullptr;
@@ -680,28 +700,29 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const uint64_t g0 = ld_relaxed_u64(gen) & 0xFFFFFFFFull;
     const uint64_t tag = kTagHigh | ((g0 + 1) & 0xFFFFFFFFull);
     PairsT<CH> P;
-    const bool bad = load_pairs<CH>(idx, n, k, E_ids, b, tokens_per_block(k, CH), P);   // in flight while zeroing
+    const bool bad = load_pairs<CH>(idx, n, k, E_ids, b, T, P);   // in flight while zeroing
     zero_words(s.wc, kWarps * E);
-    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k, CH) * mask_words(R));
+    zero_words(reinterpret_cast<int32_t *>(s.mask), T * mask_words(R));
     zero_words(s.hr, R);
-    __syncthreads();
+    lsync();
     key_and_rank<kRankKeys, CH>(idx, k, E_ids, key_div, E, s, P);
     if (with_ranks) rank_sets<CH>(k, E, R, s, P);
-    __syncthreads();
+    lsync();
     warp_offsets(E, s);
     if (with_ranks) rank_counts<CH>(k, R, s, P);
-    __syncthreads();
+    lsync();
     if (nb == 1) {   // nothing to exchange
         if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
-        if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
-        bases_and_rows<true, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
-                                        tokens_per_rank, expert_offset, max_count, dst_pos, recv_src,
-                                        status, s, P, scan_tmp);
-        return;
+        if (lsync_or(bad) && tid == 0) report(status, kErrRange);
+        bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+                                                                tokens_per_expert, tokens_per_rank, expert_offset,
+                                                                max_count, dst_pos, recv_src, status, s, P,
+                                                                scan_tmp, s_dst);
+        return true;
     }
     for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
     for (int i = tid; i < R; i += kThreads) ws_r[(int64_t)b * R + i] = s.hr[i];
-    const bool any_bad = __syncthreads_or(bad);   // also orders the workspace writes before the flag
+    const bool any_bad = lsync_or(bad);   // also orders the workspace writes before the flag
     if (tid == 0) {
         __threadfence();
         st_release_u64(flags + b, tag);
@@ -712,12 +733,30 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
 
     // every block's counts must be visible before the bases
-    if (!wait_for_flags(flags, nb, tag, status)) return;
+    if (!wait_for_flags(flags, nb, tag, status)) return false;
     if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
 
-    bases_and_rows<true, kRankKeys, CH>(ws_e, ws_r, n, k, E, R, cap, recv_rows, tokens_per_expert,
-                                    tokens_per_rank, expert_offset, max_count, dst_pos, recv_src, status,
-                                    s, P, scan_tmp);
+    bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+                                                            tokens_per_expert, tokens_per_rank, expert_offset,
+                                                            max_count, dst_pos, recv_src, status, s, P, scan_tmp,
+                                                            s_dst);
+    return true;
+}
+
+template <bool kRankKeys, int CH>
+__global__ void __launch_bounds__(kThreads)
+layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
+                    int key_div, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                    int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
+                    uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
+                    int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
+                    int32_t *__restrict__ recv_src, int64_t recv_rows, uint32_t *status) {
+    extern __shared__ __align__(16) int32_t smem_fused[];
+    __shared__ int32_t scan_tmp[32];
+    const Smem s = carve(0, smem_fused, k, E, R);
+    layout_block<kRankKeys, CH>(idx, n, k, E, R, cap, E_ids, key_div, tokens_per_block(k, CH), flags, ws_e, ws_r,
+                                tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
+                                recv_src, recv_rows, status, s, scan_tmp, nullptr);
 }
 
 template <bool kRankKeys, int CH>
@@ -890,6 +929,147 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     }
 }
 
+// ------------------------------------------- fused layout + FP8 dispatch
+//
+// Prefill-sized batches: the layout and the FP8 dispatch in one cooperative
+// launch, one CTA of 768 threads per SM.  CTA b owns tokens [b T, b T + T)
+// both as a layout block and for the dispatch.  Warps 0-7 run the layout
+// block (its barriers are hardware barrier 1, 256 threads) and keep the
+// block's receive rows in shared memory; meanwhile warps 8-23 read the CTA's
+// first B tokens and stage their FP8 codes and scales in shared memory (the
+// dispatch's HBM reads overlap the layout's latency-bound exchange; 16 warps,
+// because the per-chunk quantisation is a dependent chain that needs several
+// warps per scheduler to hide).  After a full-block barrier every thread
+// takes (token, slot) pairs and hands the staged rows to the TMA engine, one
+// bulk copy per receive row (and one per scale row), so the rest of the
+// dispatch is HBM writes only.  It runs only when a CTA's whole share fits
+// in shared memory (B >= T: at hidden 7168 up to 28 tokens per CTA, 4144 on
+// 148 SMs); a second staging round could not overlap anything and measured
+// slower than the separate kernels.
+
+constexpr int kLdThreads = 768;
+constexpr int kStageUnroll = 4;    // 16-value chunks per thread with loads in flight together
+constexpr int kLdColUnroll = 8;    // column-sum loads in flight (keeps the 768-thread kernel within 80 registers)
+
+__host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
+// Dynamic shared memory of the fused layout + dispatch kernel: the layout's
+// region, the block's receive rows (T k words), then B staged rows of h codes
+// and h / 128 fp32 scales.
+__host__ __device__ __forceinline__ size_t ld_fixed_bytes(int k, int E, int R, int T) {
+    return align16(smem_words(0, k, E, R) * sizeof(int32_t) + (size_t)T * k * sizeof(int32_t));
+}
+__host__ __device__ __forceinline__ size_t ld_row_bytes(int h) { return (size_t)h + (size_t)(h >> 7) * 4; }
+
+// Quantise `cnt` tokens starting at global token t_first into the staged rows
+// (codes qbuf[t][h], scales sbuf[t][h / 128]).  Threads [th0, th0 + nth) take
+// part (th0, nth multiples of 32); the loop is uniform over them so every lane
+// joins the shuffles.  The arithmetic is the dispatch kernel's: block absmax,
+// amax_c = max(amax, 1e-4), scale = amax_c / 448 and inv = 448 / amax_c (IEEE
+// divisions), codes = e4m3_rn_satfinite(x * inv).
+__device__ void stage_fp8_rows(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
+                               uint8_t *qbuf, float *sbuf, int th0, int nth) {
+    const int chunks = h >> 4, nblk = h >> 7;
+    const int total = cnt * chunks;    // a multiple of 8: a scale group never straddles tokens
+    const int me = (int)threadIdx.x - th0;
+    // (token, chunk) of this thread's next chunk q, advanced by nth per step
+    const int dt = nth / chunks, dc = nth - dt * chunks;
+    int t = me / chunks, c = me - t * chunks;
+    for (int base = 0; base < total; base += nth * kStageUnroll) {
+        uint4 a[kStageUnroll], b[kStageUnroll];
+        int tu[kStageUnroll], cu[kStageUnroll];
+#pragma unroll
+        for (int u = 0; u < kStageUnroll; ++u) {
+            tu[u] = t;
+            cu[u] = c;
+            a[u] = make_uint4(0, 0, 0, 0);
+            b[u] = a[u];
+            if (t < cnt) {
+                const uint16_t *src = x + (t_first + t) * h + (int64_t)c * 16;
+                a[u] = ld_nc_v4(src);
+                b[u] = ld_nc_v4(src + 8);
+            }
+            t += dt;
+            c += dc;
+            if (c >= chunks) { c -= chunks; ++t; }
+        }
+#pragma unroll
+        for (int u = 0; u < kStageUnroll; ++u) {
+            float m = absmax16(a[u], b[u]);
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            if (tu[u] < cnt) {
+                const float amax_c = fmaxf(m, 1e-4f);
+                const float scale = __fdiv_rn(amax_c, 448.0f);
+                const float inv = __fdiv_rn(448.0f, amax_c);
+                *reinterpret_cast<uint4 *>(qbuf + (size_t)tu[u] * h + (size_t)cu[u] * 16) = quant16(a[u], b[u], inv);
+                if ((cu[u] & 7) == 0) sbuf[tu[u] * nblk + (cu[u] >> 3)] = scale;
+            }
+        }
+    }
+}
+
+// Write staged tokens [tl, tl + cnt) of this CTA (staged rows 0..cnt) to their
+// receive rows: one bulk copy per (token, slot) with a row, issued by the
+// thread that takes the pair; scales by bulk copy when their row is a
+// multiple of 16 bytes and 16-byte aligned, else by plain stores.  Every
+// thread commits its own bulk group.
+__device__ void store_fp8_rows(int k, int h, int tl, int cnt, const int32_t *s_dst, const uint8_t *qbuf,
+                               const float *sbuf, uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale,
+                               bool scale_bulk) {
+    const int nblk = h >> 7;
+    const int np = cnt * k;
+    for (int p = threadIdx.x; p < np; p += blockDim.x) {
+        const int t = p / k;
+        const int32_t row = s_dst[tl * k + p];
+        if (row < 0) continue;
+        bulk_store(recv_x + (int64_t)row * h, qbuf + (size_t)t * h, (uint32_t)h);
+        if (scale_bulk) {
+            bulk_store(recv_scale + (int64_t)row * nblk, sbuf + t * nblk, (uint32_t)(nblk * 4));
+        } else {
+            for (int i = 0; i < nblk; ++i) recv_scale[(int64_t)row * nblk + i] = sbuf[t * nblk + i];
+        }
+    }
+    bulk_commit();
+}
+
+template <int CH>
+__global__ void __launch_bounds__(kLdThreads, 1)
+layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int T,
+                           int B, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                           int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
+                           uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
+                           int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
+                           int32_t *__restrict__ recv_src, int64_t recv_rows, const uint16_t *__restrict__ x,
+                           int h, uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, int scale_bulk,
+                           uint32_t *status) {
+    extern __shared__ __align__(128) int32_t smem_ld[];
+    __shared__ int32_t scan_tmp[32];
+    __shared__ int s_ok;
+    const Smem s = carve(0, smem_ld, k, E, R);
+    int32_t *s_dst = smem_ld + smem_words(0, k, E, R);
+    uint8_t *qbuf = reinterpret_cast<uint8_t *>(smem_ld) + ld_fixed_bytes(k, E, R, T);
+    float *sbuf = reinterpret_cast<float *>(qbuf + (size_t)B * h);
+    const int64_t t0 = (int64_t)blockIdx.x * T;
+    const int nt = t0 < n ? (int)(n - t0 < T ? n - t0 : T) : 0;
+    const int cnt0 = nt < B ? nt : B;   // == nt: the host launches this kernel only when B >= T
+    if (threadIdx.x < kThreads) {
+        const bool ok = layout_block<false, CH, kLdColUnroll>(idx, n, k, E, R, cap, E, E / R, T, flags, ws_e, ws_r,
+                                                tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                                                max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp,
+                                                s_dst);
+        if (threadIdx.x == 0) s_ok = ok;
+    } else {
+        stage_fp8_rows(x, h, t0, cnt0, qbuf, sbuf, kThreads, kLdThreads - kThreads);
+        fence_proxy_async();
+    }
+    __syncthreads();
+    if (!s_ok) return;   // the inter-block wait timed out (reported); nothing is written
+    store_fp8_rows(k, h, 0, cnt0, s_dst, qbuf, sbuf, recv_x, recv_scale, scale_bulk != 0);
+    bulk_wait_all();
+}
+
 // ------------------------------------------------------------------ host side
 
 std::mutex g_mu;
@@ -925,9 +1105,140 @@ bool fused_fits(int64_t n, int k, int nkeys, int R) {
     }
 }
 
+// Fused layout + FP8 dispatch: launch shape for n tokens.  T = tokens per CTA
+// (one CTA per SM, at least 64 pairs each), CH = chunks per warp of its layout
+// block, B = tokens the shared memory can stage (>= T, else ok = false and the
+// layout and the dispatch run separately).
+constexpr int kLdMaxBlocks = 256;
+struct LdShape {
+    bool ok;
+    int T, CH, B, G;
+    size_t smem;
+};
+
+LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
+    LdShape r = {false, 0, 0, 0, 0, 0};
+    int sms = device_sm_count();
+    if (num_sms > 0 && num_sms < sms) sms = num_sms;
+    if (n <= 0 || sms <= 0 || h <= 0 || h % 128 != 0) return r;
+    if (n * k < 64 * (int64_t)sms) return r;   // small batches: a few CTAs would carry the whole dispatch
+    int64_t T = (n + sms - 1) / sms;
+    const int t_min = 64 / k > 0 ? 64 / k : 1;
+    if (T < t_min) T = t_min;
+    if (T > tokens_per_block(k, kChunks)) return r;
+    const int64_t pairs = T * k;
+    r.T = (int)T;
+    r.CH = pairs <= 256 ? 1 : (pairs <= 512 ? 2 : 4);
+    r.G = (int)((n + T - 1) / T);
+    if (r.G > kLdMaxBlocks) return r;
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return r;
+    const size_t avail = optin > 1024 ? (size_t)optin - 1024 : 0;   // room for the static shared memory
+    const size_t fixed = ld_fixed_bytes(k, E, R, r.T), row = ld_row_bytes(h);
+    if (avail <= fixed) return r;
+    const size_t b = (avail - fixed) / row;
+    if (b < (size_t)r.T) return r;   // one staging round only
+    r.B = r.T;
+    r.smem = fixed + (size_t)r.B * row;
+    r.ok = true;
+    return r;
+}
+
+template <int CH>
+bool ld_launchable(const LdShape &sh) {
+    if (!ensure_smem_attr((const void *)layout_dispatch_fp8_kernel<CH>, sh.smem)) return false;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, layout_dispatch_fp8_kernel<CH>, kLdThreads, sh.smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return (int64_t)occ * device_sm_count() >= sh.G;
+}
+
+bool ld_fits(const LdShape &sh) {
+    if (!sh.ok) return false;
+    switch (sh.CH) {
+        case 1: return ld_launchable<1>(sh);
+        case 2: return ld_launchable<2>(sh);
+        default: return ld_launchable<4>(sh);
+    }
+}
+
+template <int CH>
+cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                     const uint16_t *x, int h, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                     uint8_t *in_rank, int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
+                     int32_t *recv_src, uint8_t *recv_x, float *recv_scale, void *ws, uint32_t *status,
+                     cudaStream_t stream) {
+    const WsLayout w = ws_layout_blocks(sh.G, E, R);
+    uint64_t *flags = static_cast<uint64_t *>(ws);
+    int32_t *ws_e = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.e_off);
+    int32_t *ws_r = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.r_off);
+    const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
+    const int scale_bulk = ((h >> 7) % 4 == 0) && (reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sh.G);
+    cfg.blockDim = dim3(kLdThreads);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t err = cudaLaunchKernelEx(
+        &cfg, layout_dispatch_fp8_kernel<CH>, idx, n, k, E, R, cap, sh.T, sh.B, flags, ws_e, ws_r,
+        tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src, recv_rows, x, h,
+        recv_x, recv_scale, scale_bulk, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+}
+
 }  // namespace
 
 size_t layout_workspace_bytes(int64_t n, int k, int E, int R) { return ws_layout(n, k, E, R).bytes; }
+
+size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
+    const int64_t blocks = n < 1 ? 1 : (n < kLdMaxBlocks ? n : kLdMaxBlocks);
+    const size_t fused = ws_layout_blocks(blocks, E, R).bytes, split = ws_layout(n, k, E, R).bytes;
+    return fused > split ? fused : split;
+}
+
+bool layout_dispatch_fused_fits(int64_t n, int k, int E, int R, int h, int num_sms) {
+    return ld_fits(ld_shape(n, k, E, R, h, num_sms));
+}
+
+cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
+                                      const uint16_t *x, int h, int32_t *tokens_per_expert,
+                                      int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
+                                      int32_t *max_count, int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
+                                      float *recv_scale, void *ws, int num_sms, uint32_t *status,
+                                      cudaStream_t stream) {
+    const LdShape sh = ld_shape(n, k, E, R, h, num_sms);
+    if (ld_fits(sh)) {
+        switch (sh.CH) {
+            case 1:
+                return ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                    stream);
+            case 2:
+                return ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                    stream);
+            default:
+                return ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                    stream);
+        }
+    }
+    const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
+                                        expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
+    if (st != CGL_OK) return st;
+    const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
+    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, num_sms, status, stream);
+}
 
 bool layout_needs_smem_optin(int E, int R, int k) {
     return smem_words(0, k, E, R) * sizeof(int32_t) > kSmemDefault;

@@ -288,6 +288,56 @@ cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t num_tokens, 
                                    uint32_t *status_dev, void *stream);
 
 /*
+ * Bytes of device workspace cgl_layout_dispatch_fp8 needs for these sizes
+ * (per-block counts for up to 256 blocks, or cgl_get_layout's workspace when
+ * that is larger).  Host-only; 0 for invalid sizes.
+ */
+size_t cgl_layout_dispatch_workspace_bytes(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
+
+/*
+ * Kernels cgl_layout_dispatch_fp8 launches for these sizes on the current
+ * device: 1 when the fused kernel applies, else the layout's count + 1.
+ * -1 for invalid sizes.  Host-only (queries the device once per shape).
+ */
+int cgl_layout_dispatch_kernel_count(int64_t num_tokens, int num_topk, int num_experts, int num_ranks,
+                                     int hidden, const cgl_opts *opts);
+
+/*
+ * cgl_layout_dispatch_fp8 -- cgl_get_layout and cgl_dispatch_fp8 in one call
+ * for any batch size.  Pages: the dispatch and its receive counts as for
+ * cgl_get_layout, FP8 dispatch as for cgl_dispatch_fp8 (brainleap "Day2
+ * DeepEP": the normal kernels' prefill setting, FP8 dispatch with BF16
+ * combine).  The pages have no fused form; on one GPU it lets the FP8
+ * dispatch's reads and quantisation run while the layout's blocks exchange
+ * their counts.
+ * Same outputs, ordering and errors as cgl_get_layout followed by
+ * cgl_dispatch_fp8 with the layout's dst_pos (receive rows = E*capacity when
+ * opts.capacity > 0, else num_tokens*num_topk).
+ * One cooperative kernel (one CTA of 768 threads per SM, each owning
+ * ceil(num_tokens / SMs) tokens) when every SM gets at least 64 (token, slot)
+ * pairs and a CTA's whole share of FP8 rows fits in shared memory (at hidden
+ * 7168: up to 28 tokens per CTA, 4144 tokens on 148 SMs); otherwise the
+ * layout kernel(s) then the dispatch kernel, with the same results.
+ * opts.num_sms caps the SMs used.
+ * workspace: device, >= cgl_layout_dispatch_workspace_bytes(...) bytes,
+ *   16-byte aligned, any contents (scratch for the call; overlapping calls
+ *   must not share one).
+ * Requires hidden % 128 == 0.  Alignment: x, recv_x, is_token_in_rank and the
+ * workspace 16-byte aligned; int32/fp32 arrays 4-byte (a 16-byte aligned
+ * recv_scale with hidden % 512 == 0 lets the scale rows go out as bulk copies).
+ * Device errors: as cgl_get_layout (CGL_ERANGE, CGL_ECAPACITY, CGL_ETIMEOUT
+ * for the inter-block wait, after which nothing is dispatched).
+ */
+cgl_status cgl_layout_dispatch_fp8(const int32_t *topk_idx, int64_t num_tokens, int num_topk,
+                                   int num_experts, int num_ranks, const cgl_opts *opts,
+                                   const uint16_t *x, int hidden, int32_t *tokens_per_expert,
+                                   int32_t *tokens_per_rank, uint8_t *is_token_in_rank,
+                                   int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
+                                   int32_t *recv_src, uint8_t *recv_x, float *recv_scale,
+                                   void *workspace, size_t workspace_bytes, uint32_t *status_dev,
+                                   void *stream);
+
+/*
  * cgl_combine_backward -- the gradient of cgl_combine.  Pages: combine
  * accumulates the experts' outputs (brainleap "Day2 DeepEP", "All-to-All通信");
  * this is its derivative for training.  For an output gradient g = dL/dout:

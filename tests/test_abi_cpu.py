@@ -142,3 +142,23 @@ def test_decode_dispatch_host_errors(L):
     assert L.cgl_decode_dispatch_fp8(*args(h=7000)) == cgl.EINVAL       # hidden % 128
     assert L.cgl_decode_dispatch_fp8(*args(x=p + 8)) == cgl.EALIGN
     assert L.cgl_decode_dispatch_fp8(*args(itr=p + 4)) == cgl.EALIGN
+
+
+def test_layout_dispatch_host_errors(L):
+    p = FAKE
+    ws = L.cgl_layout_dispatch_workspace_bytes(4096, 8, 256, 64)
+    assert ws >= L.cgl_layout_workspace_bytes(4096, 8, 256, 64) > 0
+    assert L.cgl_layout_dispatch_workspace_bytes(4096, 8, 256, 60) == 0     # E % R != 0
+    o = lambda cap=0, sms=0: C.byref(cgl.Opts(sms, cap))
+
+    def args(n=4096, k=8, h=7168, x=p, rs=p, wsb=ws, cap=0, w=p):
+        return (p, n, k, 256, 64, o(cap), x, h, p, p, p, p, p, p, p, p, rs, w, wsb, None, None)
+
+    assert L.cgl_layout_dispatch_fp8(*args(h=7000)) == cgl.EINVAL           # hidden % 128
+    assert L.cgl_layout_dispatch_fp8(*args(wsb=ws - 1)) == cgl.EINVAL       # workspace too small
+    assert L.cgl_layout_dispatch_fp8(*args(k=33)) == cgl.EINVAL
+    assert L.cgl_layout_dispatch_fp8(*args(cap=-1)) == cgl.EINVAL
+    assert L.cgl_layout_dispatch_fp8(*args(x=p + 8)) == cgl.EALIGN
+    assert L.cgl_layout_dispatch_fp8(*args(rs=p + 2)) == cgl.EALIGN
+    assert L.cgl_layout_dispatch_fp8(*args(w=p + 8)) == cgl.EALIGN
+    assert L.cgl_layout_dispatch_kernel_count(4096, 8, 256, 64, 7000, None) == -1
