@@ -948,7 +948,7 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 // slower than the separate kernels.
 
 constexpr int kLdThreads = 768;
-constexpr int kStageUnroll = 4;    // 16-value chunks per thread with loads in flight together
+constexpr int kStageUnroll = 2;    // 16-value chunks per batch; two batches in registers
 constexpr int kLdColUnroll = 8;    // column-sum loads in flight (keeps the 768-thread kernel within 80 registers)
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) / 16 * 16; }
@@ -967,46 +967,71 @@ __host__ __device__ __forceinline__ size_t ld_row_bytes(int h) { return (size_t)
 // joins the shuffles.  The arithmetic is the dispatch kernel's: block absmax,
 // amax_c = max(amax, 1e-4), scale = amax_c / 448 and inv = 448 / amax_c (IEEE
 // divisions), codes = e4m3_rn_satfinite(x * inv).
+struct StageBatch {
+    uint4 a[kStageUnroll], b[kStageUnroll];
+    int t[kStageUnroll], c[kStageUnroll];
+};
+
+// Issue the loads of the next kStageUnroll chunks of this thread ((t, c)
+// advanced by nth chunks per step).
+__device__ __forceinline__ void stage_load(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
+                                           int chunks, int dt, int dc, int &t, int &c, StageBatch &B) {
+#pragma unroll
+    for (int u = 0; u < kStageUnroll; ++u) {
+        B.t[u] = t;
+        B.c[u] = c;
+        B.a[u] = make_uint4(0, 0, 0, 0);
+        B.b[u] = B.a[u];
+        if (t < cnt) {
+            const uint16_t *src = x + (t_first + t) * h + (int64_t)c * 16;
+            B.a[u] = ld_nc_v4(src);
+            B.b[u] = ld_nc_v4(src + 8);
+        }
+        t += dt;
+        c += dc;
+        if (c >= chunks) { c -= chunks; ++t; }
+    }
+}
+
+__device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch &B, uint8_t *qbuf, float *sbuf) {
+    const int nblk = h >> 7;
+#pragma unroll
+    for (int u = 0; u < kStageUnroll; ++u) {
+        float m = absmax16(B.a[u], B.b[u]);
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        if (B.t[u] < cnt) {
+            const float amax_c = fmaxf(m, 1e-4f);
+            const float scale = __fdiv_rn(amax_c, 448.0f);
+            const float inv = __fdiv_rn(448.0f, amax_c);
+            *reinterpret_cast<uint4 *>(qbuf + (size_t)B.t[u] * h + (size_t)B.c[u] * 16) =
+                quant16(B.a[u], B.b[u], inv);
+            if ((B.c[u] & 7) == 0) sbuf[B.t[u] * nblk + (B.c[u] >> 3)] = scale;
+        }
+    }
+}
+
 __device__ void stage_fp8_rows(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
                                uint8_t *qbuf, float *sbuf, int th0, int nth) {
-    const int chunks = h >> 4, nblk = h >> 7;
+    const int chunks = h >> 4;
     const int total = cnt * chunks;    // a multiple of 8: a scale group never straddles tokens
     const int me = (int)threadIdx.x - th0;
-    // (token, chunk) of this thread's next chunk q, advanced by nth per step
+    // (token, chunk) of this thread's next chunk, advanced by nth per step
     const int dt = nth / chunks, dc = nth - dt * chunks;
     int t = me / chunks, c = me - t * chunks;
-    for (int base = 0; base < total; base += nth * kStageUnroll) {
-        uint4 a[kStageUnroll], b[kStageUnroll];
-        int tu[kStageUnroll], cu[kStageUnroll];
-#pragma unroll
-        for (int u = 0; u < kStageUnroll; ++u) {
-            tu[u] = t;
-            cu[u] = c;
-            a[u] = make_uint4(0, 0, 0, 0);
-            b[u] = a[u];
-            if (t < cnt) {
-                const uint16_t *src = x + (t_first + t) * h + (int64_t)c * 16;
-                a[u] = ld_nc_v4(src);
-                b[u] = ld_nc_v4(src + 8);
-            }
-            t += dt;
-            c += dc;
-            if (c >= chunks) { c -= chunks; ++t; }
-        }
-#pragma unroll
-        for (int u = 0; u < kStageUnroll; ++u) {
-            float m = absmax16(a[u], b[u]);
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            if (tu[u] < cnt) {
-                const float amax_c = fmaxf(m, 1e-4f);
-                const float scale = __fdiv_rn(amax_c, 448.0f);
-                const float inv = __fdiv_rn(448.0f, amax_c);
-                *reinterpret_cast<uint4 *>(qbuf + (size_t)tu[u] * h + (size_t)cu[u] * 16) = quant16(a[u], b[u], inv);
-                if ((cu[u] & 7) == 0) sbuf[tu[u] * nblk + (cu[u] >> 3)] = scale;
-            }
-        }
+    // two batches in registers: the next batch's loads are in flight while
+    // the current one is quantised (uniform loop: every lane joins the shuffles)
+    const int step = nth * kStageUnroll;
+    StageBatch b0, b1;
+    stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b0);
+    for (int base = 0; base < total; base += 2 * step) {
+        const bool has1 = base + step < total, has2 = base + 2 * step < total;
+        if (has1) stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b1);
+        stage_quantise(h, cnt, b0, qbuf, sbuf);
+        if (!has1) break;
+        if (has2) stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b0);
+        stage_quantise(h, cnt, b1, qbuf, sbuf);
     }
 }
 
