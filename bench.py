@@ -350,6 +350,67 @@ class GpuStep:
         e.record()
         return e
 
+    def alone_calls(self):
+        """(name, call, algorithmic bytes) of each kernel of the step, to time it alone."""
+        cgl, wl, b = self.cgl, self.wl, self.bytes
+        E, R = wl.num_experts, wl.num_ranks
+        if self.dedup:
+            lay_call = lambda: cgl.get_rank_layout(self.idx, E, R, self.rcap, workspace=self.ws, out=self.rlay,
+                                                   status=self.status)
+            dst, rows, w = self.rlay.rank_dst, self.rrows, self.w_rank
+        else:
+            lay_call = lambda: cgl.get_layout(self.idx, E, R, self.cap, workspace=self.ws, out=self.lay,
+                                              status=self.status)
+            dst, rows, w = self.lay.dst_pos, self.rows, self.w
+        calls = [("layout", lay_call, b["layout"])]
+        if wl.fp8:
+            calls.append(("dispatch_fp8", lambda: cgl.dispatch_fp8(self.x, dst, rows, recv_x=self.recv_x,
+                                                                   recv_scale=self.recv_scale, status=self.status),
+                          b["dispatch_fp8"]))
+            if self.layout_dispatch:
+                calls.append(("layout+dispatch_fp8", lambda: cgl.layout_dispatch_fp8(
+                    self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x, recv_scale=self.recv_scale,
+                    workspace=self.ws, status=self.status), b["layout"] + b["dispatch_fp8"]))
+        else:
+            calls.append(("dispatch_bf16", lambda: cgl.dispatch_bf16(self.x, dst, rows, recv_x=self.recv_x,
+                                                                     status=self.status), b["dispatch_bf16"]))
+        calls.append(("combine", lambda: cgl.combine(self.y, dst, w, out=self.out, status=self.status),
+                      b["combine"]))
+        if wl.with_grad and not self.dedup:
+            n, h, k = wl.num_tokens, wl.hidden, wl.topk
+            if self.full_backward:
+                calls.append(("combine_backward", lambda: cgl.combine_backward(
+                    self.grad, self.y, self.lay.dst_pos, self.w, grad_y=self.grad_recv, grad_w=self.grad_w,
+                    status=self.status), 2 * n * h + 4 * n * k * h + 12 * n * k))
+            else:
+                calls.append(("combine_backward", lambda: cgl.dispatch_bf16(
+                    self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv, status=self.status),
+                    b["dispatch_bf16"]))
+        return calls
+
+
+def time_alone(step: GpuStep, reps: int, peak: float):
+    """Each kernel of the step launched `reps` times back to back between two
+    CUDA events (3 launches of warm-up): µs per launch, GB/s of algorithmic
+    bytes and the fraction of the measured peak.  Inputs exceed L2."""
+    import torch
+
+    out = {}
+    for name, call, nbytes in step.alone_calls():
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / reps * 1e3
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"us": us, "bytes": nbytes, "gbs": gbs, "frac_of_peak": gbs / peak}
+    return out
+
 
 def capture_step(step: GpuStep):
     """One step's launches captured into a CUDA graph (on a side stream, after two eager runs)."""
@@ -633,6 +694,8 @@ def run_ours(args):
         barrier()
         return 0
     peak, peak_src = hbm_peak()
+    alone = time_alone(step, min(args.steps, 200), peak)
+    status_bits = sorted(set(status_bits) | set(step.cgl.status_bits(step.status)))
     kernels = {}
     for (name, launches, nbytes), t in zip(phases, per_phase):
         gbs = nbytes / (t * 1e-3) / 1e9
@@ -650,6 +713,9 @@ def run_ours(args):
     value = step.step_bytes() * world / (ms * 1e-3) / 1e9
     line.update({
         "value": value, "ms_per_step": ms, "roofline": roof, "kernels": kernels,
+        "kernels_alone": alone,
+        "kernels_alone_timing": ("each kernel of the step launched min(K, 200) times back to back between two "
+                                 "CUDA events on its stream, after 3 warm-up launches; inputs larger than L2"),
         "dispatch_plus_combine_us": sum(kernels[n]["us"] for n in kernels if n != "layout"),
         "gpu_launches": args.steps * sum(p[1] for p in phases),
         "launch": "eager" if args.no_graph else "CUDA graph of one step, replayed K times (e2e and per-kernel passes eager)",
