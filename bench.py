@@ -708,7 +708,11 @@ def run_ours(args):
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
             "bytes_per_launch": kernels[dom]["bytes"],
-            "timing": "CUDA events around each launch in the instrumented pass (launch gap included)"}
+            "achieved_alone": alone[dom]["gbs"] if dom in alone else None,
+            "frac_alone": alone[dom]["frac_of_peak"] if dom in alone else None,
+            "timing": ("achieved / frac: CUDA events around each launch in the instrumented pass (launch gap "
+                       "included); achieved_alone / frac_alone: the same kernel launched back to back "
+                       "(kernels_alone)")}
     line = base_line(args, wl, world)
     value = step.step_bytes() * world / (ms * 1e-3) / 1e9
     line.update({
