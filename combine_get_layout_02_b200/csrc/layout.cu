@@ -813,6 +813,97 @@ layout_rows_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int
                                      s, P, scan_tmp);
 }
 
+// ---------------------------------------------------------- cluster layout
+//
+// Small batches (2 to 8 blocks of one chunk per warp: up to 256 tokens at
+// top-8): the blocks run as one thread-block cluster and exchange their
+// counts through distributed shared memory instead of the workspace.  After a
+// hardware cluster barrier every CTA reads the other CTAs' per-key counts
+// (mapa + ld.shared::cluster) for its prefix over earlier CTAs and the
+// totals; CTA 0 also sums the distinct-token counts per rank.  A CTA arrives
+// at a second cluster barrier once its peer reads are done and waits on it
+// only before it exits, so no CTA's shared memory goes away while a peer may
+// still read it.  No global round trip between the phases.
+
+constexpr int kMaxClusterCtas = 8;   // portable cluster size
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The int32 at the same shared-memory offset as `local` in cluster CTA `rank`.
+__device__ __forceinline__ int32_t ld_cluster_peer(const int32_t *local, uint32_t rank) {
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(local);
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+// Grid = exactly one cluster of C = gridDim.x CTAs (cluster rank = blockIdx.x);
+// CTA b owns tokens [b T, b T + T), T = tokens_per_block(k, 1).
+template <bool kRankKeys>
+__global__ void __launch_bounds__(kThreads)
+layout_cluster_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
+                      int key_div, int32_t *__restrict__ tokens_per_key, int32_t *__restrict__ tokens_per_rank,
+                      uint8_t *__restrict__ in_rank, int32_t *__restrict__ key_offset,
+                      int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
+                      int32_t *__restrict__ recv_src, int64_t recv_rows, uint32_t *status) {
+    extern __shared__ __align__(16) int32_t smem_cl[];
+    __shared__ int32_t scan_tmp[32];
+    const Smem s = carve(0, smem_cl, k, E, R);
+    const int tid = threadIdx.x;
+    const int C = gridDim.x, b = blockIdx.x;
+    const int T = tokens_per_block(k, 1);
+    const bool with_ranks = in_rank != nullptr;
+    PairsT<1> P;
+    const bool bad = load_pairs<1>(idx, n, k, E_ids, b, T, P);   // in flight while zeroing
+    zero_words(s.wc, kWarps * E);
+    zero_words(reinterpret_cast<int32_t *>(s.mask), T * mask_words(R));
+    zero_words(s.hr, R);
+    lsync();
+    key_and_rank<kRankKeys, 1>(idx, k, E_ids, key_div, E, s, P);
+    if (with_ranks) rank_sets<1>(k, E, R, s, P);
+    lsync();
+    warp_offsets(E, s);
+    if (with_ranks) rank_counts<1>(k, R, s, P);
+    if (bad) report(status, kErrRange);
+    cluster_arrive_release();   // this CTA's counts are final; its rank rows go out while peers catch up
+    if (with_ranks) write_rank_rows<1>(R, in_rank, s, P);
+    cluster_wait_acquire();     // every CTA's counts are visible cluster-wide
+    for (int e = tid; e < E; e += kThreads) {
+        int32_t tot = 0, pre = 0;
+#pragma unroll
+        for (int c = 0; c < kMaxClusterCtas; ++c) {
+            if (c < C) {
+                const int32_t v = ld_cluster_peer(s.he + e, (uint32_t)c);
+                tot += v;
+                pre += c < b ? v : 0;
+            }
+        }
+        s.total[e] = tot;
+        s.base[e] = pre;
+    }
+    if (b == 0 && with_ranks && tokens_per_rank != nullptr) {
+        for (int r = tid; r < R; r += kThreads) {
+            int32_t tot = 0;
+#pragma unroll
+            for (int c = 0; c < kMaxClusterCtas; ++c)
+                if (c < C) tot += ld_cluster_peer(s.hr + r, (uint32_t)c);
+            tokens_per_rank[r] = tot;
+        }
+    }
+    cluster_arrive_release();   // this CTA reads no peer shared memory after this point
+    lsync();
+    bases_and_rows<true, kRankKeys, 1, true>(nullptr, nullptr, n, k, E, R, cap, recv_rows, tokens_per_key,
+                                             nullptr, key_offset, max_count, dst_pos, recv_src, status, s, P,
+                                             scan_tmp);
+    cluster_wait_acquire();     // the peers have finished reading this CTA's shared memory
+}
+
 // Fused decode path: the layout and the FP8 dispatch of a small batch (at most
 // 1024 (token, slot) pairs) in one launch, no workspace.  Every CTA computes the
 // whole layout in shared memory (one layout block's work, so no inter-block
@@ -1119,6 +1210,44 @@ int fused_capacity() {
     return slot > 0 ? slot * device_sm_count() : 0;
 }
 
+int g_cluster_ok[2][64][kMaxClusterCtas + 1] = {{{0}}};   // per mode, device, size: 1 ok, -1 no
+
+// CTAs of the cluster layout for n tokens (2..8 blocks of tokens_per_block(k, 1)
+// tokens whose shared memory needs no opt-in and that the device can
+// schedule as one cluster; queried once per size), else 0.
+template <bool kRankKeys>
+int cluster_ctas_for(int64_t n, int k, int nkeys, int R) {
+    const int T = tokens_per_block(k, 1);
+    const int64_t C = (n + T - 1) / T;
+    if (C < 2 || C > kMaxClusterCtas) return 0;
+    const size_t smem = smem_words(0, k, nkeys, R) * sizeof(int32_t);
+    if (smem > kSmemDefault) return 0;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(g_mu);
+    int &ok = g_cluster_ok[kRankKeys ? 1 : 0][dev][C];
+    if (ok == 0) {
+        ok = -1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemDefault;   // the most this path uses
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, layout_cluster_kernel<kRankKeys>, &cfg) == cudaSuccess &&
+            clusters >= 1)
+            ok = 1;
+        cudaGetLastError();   // a refused query must not linger as a sticky launch error
+    }
+    return ok == 1 ? (int)C : 0;
+}
+
 template <bool kRankKeys>
 bool fused_fits(int64_t n, int k, int nkeys, int R) {
     const WsLayout w = ws_layout(n, k, nkeys, R);
@@ -1324,6 +1453,27 @@ cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, i
                               int32_t *tokens_per_key, int32_t *tokens_per_rank, uint8_t *in_rank,
                               int32_t *key_offset, int32_t *max_count, int32_t *dst_pos,
                               int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
+    const int nkeys = kRankKeys ? R : E_ids;
+    const int C = cluster_ctas_for<kRankKeys>(n, k, nkeys, R);
+    if (C > 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem_words(0, k, nkeys, R) * sizeof(int32_t);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const int64_t recv_rows = cap > 0 ? (int64_t)nkeys * cap : n * k;
+        const cudaError_t err = cudaLaunchKernelEx(&cfg, layout_cluster_kernel<kRankKeys>, idx, n, k, nkeys, R, cap,
+                                                   E_ids, E_ids / R, tokens_per_key, tokens_per_rank, in_rank,
+                                                   key_offset, max_count, dst_pos, recv_src, recv_rows, status);
+        return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    }
     switch (layout_chunks(n, k)) {
         case 1:
             return launch_layout_ch<kRankKeys, 1>(idx, n, k, E_ids, R, cap, tokens_per_key, tokens_per_rank,

@@ -66,6 +66,21 @@ def test_layout_block_size_boundaries(oracle_mod, n, k):
     run_both(oracle_mod, idx, E, R, max(1, int(lay.max_count.item()) - 3))   # a few copies over capacity
 
 
+@pytest.mark.parametrize("n,k,E,R", [(33, 8, 256, 64), (64, 8, 256, 32), (100, 8, 256, 64), (200, 8, 256, 64),
+                                     (256, 8, 256, 64), (170, 3, 64, 8), (96, 6, 96, 12), (130, 4, 16, 4)])
+def test_layout_cluster_sizes(oracle_mod, n, k, E, R):
+    """Batches of 2 to 8 one-chunk blocks (the thread-block-cluster path): duplicates
+    inside tokens, masked and bad ids, compact and padded with overflow."""
+    rng = np.random.default_rng(n * 7 + k)
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    idx[rng.random((n, k)) < 0.05] = -1
+    idx[rng.random((n, k)) < 0.01] = E
+    lay, _ = run_both(oracle_mod, idx, E, R, 0)
+    mc = int(lay.max_count.item())
+    run_both(oracle_mod, idx, E, R, max(1, mc - 2))
+    run_both(oracle_mod, idx, E, R, mc + 1)
+
+
 def test_layout_duplicates_bad_ids_and_overflow(oracle_mod):
     rng = np.random.default_rng(42)
     n, k, E, R = 700, 8, 16, 4

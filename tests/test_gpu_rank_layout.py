@@ -128,3 +128,14 @@ def test_dedup_path_equals_expert_path_normwise(oracle_mod):
     a = W.bf16_bits_to_f32(out).astype(np.float64)
     b = W.bf16_bits_to_f32(ref).astype(np.float64)
     assert np.linalg.norm(a - b) <= 2.0 ** -7 * np.linalg.norm(b)
+
+
+@pytest.mark.parametrize("n,k,E,R", [(40, 8, 256, 64), (200, 8, 256, 32), (170, 3, 64, 8), (130, 6, 96, 12)])
+def test_rank_layout_cluster_sizes(oracle_mod, n, k, E, R):
+    """Rank keys on the thread-block-cluster path (2 to 8 one-chunk blocks)."""
+    rng = np.random.default_rng(n + 13 * k)
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)        # repeated ranks and experts inside tokens
+    idx[rng.random((n, k)) < 0.05] = -1
+    idx[rng.random((n, k)) < 0.01] = E + 2
+    rl, ref = run_both(oracle_mod, idx, E, R)
+    run_both(oracle_mod, idx, E, R, max(1, ref.max_count - 1))
