@@ -40,8 +40,10 @@
 //                   Block 0 writes the global counts, offsets and max.
 //   rows          : row = expert base + earlier blocks + warp offset + rank.
 //
-// Launch shapes.  With one block (up to 1024 pairs, e.g. 128 decode tokens at
-// k = 8) the block's own counts are the totals and nothing is exchanged.
+// Launch shapes.  Batches of 2 to 8 one-chunk blocks (up to 256 tokens at
+// k = 8, e.g. 128 decode tokens as 4 CTAs) run as one thread-block cluster
+// that exchanges counts through distributed shared memory (below).  With one
+// block the block's own counts are the totals and nothing is exchanged.
 // When every block fits on the GPU at once, one cooperative kernel does
 // everything and the blocks exchange their counts through the workspace: each
 // block writes its row, then release-stores this launch's 64-bit tag into its
