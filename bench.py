@@ -44,7 +44,8 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {
     "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
     "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
-    "layout": {"bytes": 206080, "src_sha": "2315501c74f4a785"},
+    "layout": {"bytes": 206080, "src_sha": "2c671e30ceab350f"},
+    "layout+dispatch_fp8": {"bytes": 244837376, "src_sha": "2c671e30ceab350f"},
 }
 
 
@@ -718,7 +719,8 @@ def run_ours(args):
                          "gbs": gbs, "frac_of_peak": gbs / peak}
     dom = max(phases, key=lambda p: p[2])[0]
     src = {"combine": "combine.cu", "dispatch_fp8": "dispatch.cu", "dispatch_bf16": "dispatch.cu",
-           "layout": "layout.cu", "combine_backward": "combine_backward.cu"}.get(dom, "layout.cu")
+           "layout": "layout.cu", "layout+dispatch_fp8": "layout.cu",
+           "combine_backward": "combine_backward.cu"}.get(dom, "layout.cu")
     roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
