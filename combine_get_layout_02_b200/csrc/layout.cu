@@ -1266,6 +1266,21 @@ bool fused_fits(int64_t n, int k, int nkeys, int R) {
 // block, B = tokens the shared memory can stage (>= T, else ok = false and the
 // layout and the dispatch run separately).
 constexpr int kLdMaxBlocks = 256;
+
+int g_optin_smem[64] = {0};   // per device: largest dynamic shared memory a block may opt in to
+
+int optin_smem_bytes() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_optin_smem[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+        g_optin_smem[dev] = v > 0 ? v : -1;
+    }
+    return g_optin_smem[dev];
+}
+
 struct LdShape {
     bool ok;
     int T, CH, B, G;
@@ -1287,10 +1302,8 @@ LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
     r.CH = pairs <= 256 ? 1 : (pairs <= 512 ? 2 : 4);
     r.G = (int)((n + T - 1) / T);
     if (r.G > kLdMaxBlocks) return r;
-    int dev = 0, optin = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-        return r;
+    const int optin = optin_smem_bytes();
+    if (optin <= 0) return r;
     const size_t avail = optin > 1024 ? (size_t)optin - 1024 : 0;   // room for the static shared memory
     const size_t fixed = ld_fixed_bytes(k, E, R, r.T), row = ld_row_bytes(h);
     if (avail <= fixed) return r;
@@ -1302,14 +1315,35 @@ LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
     return r;
 }
 
+// CTAs per SM of the fused kernel at this shared memory, cached per device, CH
+// and size (the shared memory only takes a few values: one per tokens per CTA).
+struct LdOcc {
+    int dev, ch;
+    size_t smem;
+    int occ;
+};
+LdOcc g_ld_occ[64];
+int g_ld_occ_n = 0;
+
 template <int CH>
 bool ld_launchable(const LdShape &sh) {
     if (!ensure_smem_attr((const void *)layout_dispatch_fp8_kernel<CH>, sh.smem)) return false;
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, layout_dispatch_fp8_kernel<CH>, kLdThreads, sh.smem) !=
-        cudaSuccess) {
-        cudaGetLastError();
-        return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    int occ = -1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (int i = 0; i < g_ld_occ_n; ++i)
+            if (g_ld_occ[i].dev == dev && g_ld_occ[i].ch == CH && g_ld_occ[i].smem == sh.smem) occ = g_ld_occ[i].occ;
+    }
+    if (occ < 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, layout_dispatch_fp8_kernel<CH>, kLdThreads,
+                                                          sh.smem) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_ld_occ_n < 64) g_ld_occ[g_ld_occ_n++] = {dev, CH, sh.smem, occ};
     }
     return (int64_t)occ * device_sm_count() >= sh.G;
 }
