@@ -1032,9 +1032,9 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 // first B tokens and stage their FP8 codes and scales in shared memory (the
 // dispatch's HBM reads overlap the layout's latency-bound exchange; 16 warps,
 // because the per-chunk quantisation is a dependent chain that needs several
-// warps per scheduler to hide).  After a full-block barrier every thread
-// takes (token, slot) pairs and hands the staged rows to the TMA engine, one
-// bulk copy per receive row (and one per scale row), so the rest of the
+// warps per scheduler to hide).  After a full-block barrier the lanes of
+// warp 0 take (token, slot) pairs and hand the staged rows to the TMA engine,
+// one bulk copy per receive row (and one per scale row), so the rest of the
 // dispatch is HBM writes only.  It runs only when a CTA's whole share fits
 // in shared memory (B >= T: at hidden 7168 up to 28 tokens per CTA, 4144 on
 // 148 SMs); a second staging round could not overlap anything and measured
@@ -1130,15 +1130,17 @@ __device__ void stage_fp8_rows(const uint16_t *__restrict__ x, int h, int64_t t_
 
 // Write staged tokens [tl, tl + cnt) of this CTA (staged rows 0..cnt) to their
 // receive rows: one bulk copy per (token, slot) with a row, issued by the
-// thread that takes the pair; scales by bulk copy when their row is a
-// multiple of 16 bytes and 16-byte aligned, else by plain stores.  Every
-// thread commits its own bulk group.
+// lanes of warp 0 (measured ~1% faster than spreading the issue over every
+// thread); scales by bulk copy when their row is a multiple of 16 bytes and
+// 16-byte aligned, else by plain stores.  Each issuing lane commits its own
+// bulk group.
 __device__ void store_fp8_rows(int k, int h, int tl, int cnt, const int32_t *s_dst, const uint8_t *qbuf,
                                const float *sbuf, uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale,
                                bool scale_bulk) {
     const int nblk = h >> 7;
     const int np = cnt * k;
-    for (int p = threadIdx.x; p < np; p += blockDim.x) {
+    if (threadIdx.x >= 32) return;
+    for (int p = threadIdx.x; p < np; p += 32) {
         const int t = p / k;
         const int32_t row = s_dst[tl * k + p];
         if (row < 0) continue;
