@@ -41,13 +41,13 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per launch read by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the kernels at the 4096-token prefill shape, with the sha256 of the kernel
 # source they were taken on; a changed source reports traffic null.  (The
-# layout records were carried over one edit of layout.cu that touched host
-# code only: a cache of the fused kernel's occupancy query.)
+# "layout" record was carried over edits of layout.cu that did not touch
+# layout_fused_kernel: host-side caches and the fused dispatch's store loop.)
 NCU_TRAFFIC = {
     "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
     "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
-    "layout": {"bytes": 206080, "src_sha": "14f02c3a04ff21a7"},
-    "layout+dispatch_fp8": {"bytes": 244837376, "src_sha": "14f02c3a04ff21a7"},
+    "layout": {"bytes": 206080, "src_sha": "f22f0a4280d260df"},
+    "layout+dispatch_fp8": {"bytes": 246364416, "src_sha": "f22f0a4280d260df"},
 }
 
 
