@@ -8,10 +8,13 @@
 //
 // Work unit: a CTA owns one token at a time (persistent over tokens), one
 // thread per 16 hidden values (every 512th chunk when the row is longer).  Per
-// batch of 8 slots a thread loads its 32 bytes of g and of each slot's y row
+// batch of 4 slots a thread loads its 32 bytes of g and of each slot's y row
 // (all loads in flight before any math), writes
-// the 8 scaled gradient chunks with 16-byte stores and keeps 8 partial dot
-// products (fused multiply-adds over its values in order).  The block then
+// the 4 scaled gradient chunks with 16-byte stores and keeps 4 partial dot
+// products (fused multiply-adds over its values in order).  Batches of 4 keep
+// the kernel at 64 registers, so two CTAs share an SM and one's loads cover
+// the other's block reduction (batches of 8 needed 117 registers: one CTA
+// per SM, idle HBM during every reduction).  The block then
 // reduces the partial dots with xor-shuffles and one pass over the warps in
 // warp order, so grad_w does not depend on timing.  Launches use programmatic
 // dependent launch.
@@ -22,11 +25,11 @@ namespace cgl {
 
 namespace {
 
-constexpr int kBatch = 8;                // slots whose rows are loaded together
+constexpr int kBatch = 4;                // slots whose rows are loaded together
 constexpr int kThreadsPerSM = 1024;      // CTAs per SM = this / block size (at least 1)
 constexpr int kMaxThreads = 512;         // larger rows loop: each thread takes every 512th chunk
 
-__global__ void __launch_bounds__(kMaxThreads)
+__global__ void __launch_bounds__(kMaxThreads, 2)
 combine_backward_kernel(const uint16_t *__restrict__ g, const uint16_t *__restrict__ y, int64_t recv_rows,
                         const int32_t *__restrict__ dst_pos, const float *__restrict__ w, int64_t n, int h,
                         int k, uint16_t *__restrict__ grad_y, float *__restrict__ grad_w, uint32_t *status) {
