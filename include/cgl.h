@@ -84,9 +84,9 @@ size_t cgl_layout_workspace_bytes(int64_t num_tokens, int num_topk, int num_expe
 
 /*
  * Number of kernels cgl_get_layout launches for these sizes on the current
- * device: 1 (one cooperative kernel) when all its blocks fit on the GPU at
- * once, else 2.  -1 for invalid sizes.  Host-only (queries the device's
- * occupancy once).
+ * device: 1 (one thread-block cluster for 2 to 8 small blocks, else one
+ * cooperative kernel) when all its blocks fit on the GPU at once, else 2.
+ * -1 for invalid sizes.  Host-only (queries the device's occupancy once).
  */
 int cgl_layout_kernel_count(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
 
