@@ -1385,7 +1385,10 @@ cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, in
         &cfg, layout_dispatch_fp8_kernel<CH>, idx, n, k, E, R, cap, sh.T, sh.B, flags, ws_e, ws_r,
         tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src, recv_rows, x, h,
         recv_x, recv_scale, scale_bulk, status);
-    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    if (err == cudaSuccess) return CGL_OK;
+    if (err != cudaErrorCooperativeLaunchTooLarge) return CGL_ECUDA;
+    cudaGetLastError();   // fewer SMs free than the occupancy query counted: the caller splits the work
+    return CGL_ENOTIMPL;
 }
 
 }  // namespace
@@ -1410,20 +1413,24 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       cudaStream_t stream) {
     const LdShape sh = ld_shape(n, k, E, R, h, num_sms);
     if (ld_fits(sh)) {
+        cgl_status st = CGL_ECUDA;
         switch (sh.CH) {
             case 1:
-                return ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                    stream);
+                st = ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                  stream);
+                break;
             case 2:
-                return ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                    stream);
+                st = ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                  stream);
+                break;
             default:
-                return ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                    stream);
+                st = ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
+                                  stream);
         }
+        if (st != CGL_ENOTIMPL) return st;   // CGL_ENOTIMPL: the cooperative launch was refused
     }
     const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
                                         expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
@@ -1466,7 +1473,9 @@ cgl_status launch_layout_ch(const int32_t *idx, int64_t n, int k, int E_ids, int
             &cfg, layout_fused_kernel<kRankKeys, CH>, idx, n, k, E, R, cap, E_ids, key_div, flags, ws_e, ws_r,
             tokens_per_key, tokens_per_rank, in_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
             status);
-        return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+        if (err == cudaSuccess) return CGL_OK;
+        if (err != cudaErrorCooperativeLaunchTooLarge) return CGL_ECUDA;
+        cudaGetLastError();   // fewer SMs free than the occupancy query counted: use the two kernels
     }
 
     const size_t smem1 = smem_words(1, k, E, R) * sizeof(int32_t);
