@@ -43,13 +43,11 @@ FALLBACK_HBM_GBS = 6650.0
 # source they were taken on; a changed source reports traffic null.  (The
 # "layout" record was carried over edits of layout.cu that did not touch
 # layout_fused_kernel: host-side caches, launch fallbacks and the fused
-# dispatch's store loop; the "layout+dispatch_fp8" record over the last two
-# host-only edits.)
+# dispatch's store loop and count-row format.)
 NCU_TRAFFIC = {
     "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
     "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
-    "layout": {"bytes": 206080, "src_sha": "9de58f9fecf8addb"},
-    "layout+dispatch_fp8": {"bytes": 246364416, "src_sha": "9de58f9fecf8addb"},
+    "layout": {"bytes": 206080, "src_sha": "8cdb38836f26e97a"},
 }
 
 

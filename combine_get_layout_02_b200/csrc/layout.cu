@@ -484,6 +484,77 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
     lsync();
 }
 
+// The same over a table of 16-bit counts (a block's count per key is at most
+// its 1024 pairs), ncols a multiple of 8: one 16-byte load carries 8 columns,
+// so the all-blocks read moves half the bytes of the 32-bit table.
+template <bool kCoherent>
+__device__ __forceinline__ uint4 ld_col8_u16(const uint16_t *p) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+    return kCoherent ? __ldcg(q) : __ldg(q);
+}
+
+template <bool kCoherent, int U = kColUnroll>
+__device__ void column_sums_u16(const uint16_t *t, int nb, int ncols, int upto, int32_t *out_tot,
+                                int32_t *out_pre, int32_t *part) {
+    const int tid = threadIdx.x;
+    const int nq = ncols / 8;                        // 16-byte loads per row
+    int G = nq >= kThreads ? 1 : kThreads / nq;
+    if (2 * G * ncols > kPartWords) G = kPartWords / (2 * ncols);
+    if (G < 1) G = 1;
+    const int q0 = G > 1 ? tid % nq : tid;
+    const int g = G > 1 ? tid / nq : 0;
+    const int qstep = G > 1 ? nq : kThreads;
+    if (g < G) {
+        for (int q = q0; q < nq; q += qstep) {
+            int32_t tot[8] = {0, 0, 0, 0, 0, 0, 0, 0}, pre[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            for (int r0 = g; r0 < nb; r0 += G * U) {
+                uint4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int r = r0 + u * G;
+                    v[u] = r < nb ? ld_col8_u16<kCoherent>(t + (int64_t)r * ncols + q * 8) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int32_t below = r0 + u * G < upto ? 1 : 0;
+                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int32_t lo = (int32_t)(w[i] & 0xFFFFu), hi = (int32_t)(w[i] >> 16);
+                        tot[2 * i] += lo;
+                        tot[2 * i + 1] += hi;
+                        pre[2 * i] += below * lo;
+                        pre[2 * i + 1] += below * hi;
+                    }
+                }
+            }
+            for (int c = 0; c < 8; ++c) {
+                const int col = q * 8 + c;
+                if (G > 1) {
+                    part[g * ncols + col] = tot[c];
+                    part[(G + g) * ncols + col] = pre[c];
+                } else {
+                    out_tot[col] = tot[c];
+                    if (out_pre) out_pre[col] = pre[c];
+                }
+            }
+        }
+    }
+    if (G > 1) {
+        lsync();
+        for (int col = tid; col < ncols; col += kThreads) {
+            int32_t a = 0, b = 0;
+            for (int gg = 0; gg < G; ++gg) {
+                a += part[gg * ncols + col];
+                b += part[(G + gg) * ncols + col];
+            }
+            out_tot[col] = a;
+            if (out_pre) out_pre[col] = b;
+        }
+    }
+    lsync();
+}
+
 // Exclusive scan of v[0..n) in shared memory (n <= kMaxExperts) into out[];
 // returns the total.  All threads of the block must call it.
 template <int NT = kThreads>
@@ -524,7 +595,7 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
 // Bases, the global outputs (block 0) and the rows of the block's pairs.
 // kTotalsGiven: s.total / s.base (copies in earlier blocks) are already set.
 template <bool kCoherent, bool kRankKeys, int CH = kChunks, bool kTotalsGiven = false, int NT = kThreads,
-          int U = kColUnroll>
+          int U = kColUnroll, bool kU16 = false>
 __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t n, int k, int E, int R,
                                int cap, int64_t recv_rows, int32_t *__restrict__ tokens_per_expert,
                                int32_t *__restrict__ tokens_per_rank, int32_t *__restrict__ expert_offset,
@@ -556,7 +627,11 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         }
         lsync();
     } else {
-        column_sums<kCoherent, U>(ws_e, nb, E, b, s.total, s.base, s.part);
+        if constexpr (kU16)
+            column_sums_u16<kCoherent, U>(reinterpret_cast<const uint16_t *>(ws_e), nb, E, b, s.total, s.base,
+                                          s.part);
+        else
+            column_sums<kCoherent, U>(ws_e, nb, E, b, s.total, s.base, s.part);
     }
     if (rank_sums) {
         for (int r = rcol; r < R; r += nb * (NT / 32)) {   // warp-uniform
@@ -682,7 +757,7 @@ __device__ void zero_words(int32_t *p, int n) {
 // for the key transform; in_rank == nullptr skips the rank sets (rank mode).
 // s_dst (optional, shared memory, T k words) also receives the block's rows.
 // Returns false (the whole group of 256) when the inter-block wait timed out.
-template <bool kRankKeys, int CH, int U = kColUnroll>
+template <bool kRankKeys, int CH, int U = kColUnroll, bool kU16 = false>
 __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
                              int key_div, int T, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
                              int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
@@ -716,13 +791,18 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     if (nb == 1) {   // nothing to exchange
         if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
         if (lsync_or(bad) && tid == 0) report(status, kErrRange);
-        bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+        bases_and_rows<true, kRankKeys, CH, false, kThreads, U, kU16>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
                                                                 tokens_per_expert, tokens_per_rank, expert_offset,
                                                                 max_count, dst_pos, recv_src, status, s, P,
                                                                 scan_tmp, s_dst);
         return true;
     }
-    for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
+    if constexpr (kU16) {   // 16-bit count rows (E % 8 == 0; counts <= 1024)
+        uint16_t *row = reinterpret_cast<uint16_t *>(ws_e) + (int64_t)b * E;
+        for (int i = tid; i < E; i += kThreads) row[i] = (uint16_t)s.he[i];
+    } else {
+        for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
+    }
     for (int i = tid; i < R; i += kThreads) ws_r[(int64_t)b * R + i] = s.hr[i];
     const bool any_bad = lsync_or(bad);   // also orders the workspace writes before the flag
     if (tid == 0) {
@@ -738,7 +818,7 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     if (!wait_for_flags(flags, nb, tag, status)) return false;
     if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
 
-    bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+    bases_and_rows<true, kRankKeys, CH, false, kThreads, U, kU16>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
                                                             tokens_per_expert, tokens_per_rank, expert_offset,
                                                             max_count, dst_pos, recv_src, status, s, P, scan_tmp,
                                                             s_dst);
@@ -1175,7 +1255,7 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
     const int nt = t0 < n ? (int)(n - t0 < T ? n - t0 : T) : 0;
     const int cnt0 = nt < B ? nt : B;   // == nt: the host launches this kernel only when B >= T
     if (threadIdx.x < kThreads) {
-        const bool ok = layout_block<false, CH, kLdColUnroll>(idx, n, k, E, R, cap, E, E / R, T, flags, ws_e, ws_r,
+        const bool ok = layout_block<false, CH, kLdColUnroll, true>(idx, n, k, E, R, cap, E, E / R, T, flags, ws_e, ws_r,
                                                 tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
                                                 max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp,
                                                 s_dst);
@@ -1295,6 +1375,7 @@ LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
     if (num_sms > 0 && num_sms < sms) sms = num_sms;
     if (n <= 0 || sms <= 0 || h <= 0 || h % 128 != 0) return r;
     if (n * k < 64 * (int64_t)sms) return r;   // small batches: a few CTAs would carry the whole dispatch
+    if (E % 8 != 0) return r;                   // its count rows are 16-bit, 8 per 16-byte load
     int64_t T = (n + sms - 1) / sms;
     const int t_min = 64 / k > 0 ? 64 / k : 1;
     if (T < t_min) T = t_min;

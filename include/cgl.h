@@ -315,7 +315,7 @@ int cgl_layout_dispatch_kernel_count(int64_t num_tokens, int num_topk, int num_e
  * opts.capacity > 0, else num_tokens*num_topk).
  * One cooperative kernel (one CTA of 768 threads per SM, each owning
  * ceil(num_tokens / SMs) tokens) when every SM gets at least 64 (token, slot)
- * pairs and a CTA's whole share of FP8 rows fits in shared memory (at hidden
+ * pairs, num_experts % 8 == 0 and a CTA's whole share of FP8 rows fits in shared memory (at hidden
  * 7168: up to 28 tokens per CTA, 4144 tokens on 148 SMs); otherwise the
  * layout kernel(s) then the dispatch kernel, with the same results.
  * opts.num_sms caps the SMs used.
