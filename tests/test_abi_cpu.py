@@ -162,3 +162,13 @@ def test_layout_dispatch_host_errors(L):
     assert L.cgl_layout_dispatch_fp8(*args(rs=p + 2)) == cgl.EALIGN
     assert L.cgl_layout_dispatch_fp8(*args(w=p + 8)) == cgl.EALIGN
     assert L.cgl_layout_dispatch_kernel_count(4096, 8, 256, 64, 7000, None) == -1
+
+
+def test_layout_dispatch_workspace_covers_the_split_path(L):
+    # the combined call falls back to cgl_get_layout + cgl_dispatch_fp8, so its
+    # workspace must be at least the layout's for every size
+    for n in (0, 1, 31, 32, 33, 127, 128, 129, 256, 257, 1000, 4095, 4096, 4097, 8193, 16384, 70000):
+        for k, E, R in ((8, 256, 64), (1, 4, 2), (6, 96, 12), (32, 1024, 64)):
+            a = L.cgl_layout_dispatch_workspace_bytes(n, k, E, R)
+            b = L.cgl_layout_workspace_bytes(n, k, E, R)
+            assert a >= b > 0, (n, k, E, R, a, b)
