@@ -177,3 +177,43 @@ def test_rank_layout_invariants(oracle_mod, name):
         seg = RL.recv_token[RL.rank_offset[r]:RL.rank_offset[r + 1]]
         assert np.all(np.diff(seg) > 0) and np.all((ranks[seg] == r).any(axis=1))
     assert np.all(RL.recv_token[rows:] == -1)
+
+
+# Property-based pin: hypothesis draws tiny shapes and id tables (duplicates,
+# masked and out-of-range ids, compact or padded with any capacity) and the
+# oracle must equal the brute force exactly, for expert and for rank keys.
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+
+@st.composite
+def _tables(draw):
+    E = draw(st.sampled_from([1, 2, 4, 6, 8, 12]))
+    R = draw(st.sampled_from([r for r in (1, 2, 3, 4, 6, 12) if r <= E and E % r == 0]))
+    k = draw(st.integers(1, 5))
+    n = draw(st.integers(0, 24))
+    ids = draw(st.lists(st.lists(st.integers(-3, E + 2), min_size=k, max_size=k), min_size=n, max_size=n))
+    cap = draw(st.integers(0, 6))
+    idx = np.array(ids, dtype=np.int32).reshape(n, k)
+    return idx, E, R, cap
+
+
+@settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(_tables())
+def test_layout_equals_brute_force_property(oracle_mod, table):
+    idx, E, R, cap = table
+    _compare_to_brute(oracle_mod, idx, E, R, cap)
+
+
+@settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(_tables())
+def test_rank_layout_equals_brute_force_property(oracle_mod, table):
+    idx, E, R, cap = table
+    L = oracle_mod.get_rank_layout(idx, E, R, cap)
+    B = brute.rank_layout(idx.tolist(), E, R, cap)
+    assert L.tokens_per_rank.tolist() == B["tokens_per_rank"]
+    assert L.rank_offset.tolist() == B["rank_offset"]
+    assert L.max_count == B["max_count"]
+    assert L.rank_dst.tolist() == B["rank_dst"]
+    assert L.recv_token.tolist() == B["recv_token"]
+    assert bool(L.flags & oracle_mod.FLAG_CAPACITY) == B["capacity_error"]
