@@ -172,3 +172,11 @@ def test_layout_dispatch_workspace_covers_the_split_path(L):
             a = L.cgl_layout_dispatch_workspace_bytes(n, k, E, R)
             b = L.cgl_layout_workspace_bytes(n, k, E, R)
             assert a >= b > 0, (n, k, E, R, a, b)
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    # no CPU or PyTorch fallback: a missing libcgl.so is an error at the first call
+    monkeypatch.setattr(cgl, "_lib", None)
+    monkeypatch.setattr(cgl, "LIB_PATH", str(tmp_path / "libcgl.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        cgl.layout_workspace_bytes(4096, 8, 256, 64)
