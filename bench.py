@@ -449,6 +449,47 @@ def capture_step(step: GpuStep):
     return g
 
 
+def time_phase_graphs(step: GpuStep, steps: int):
+    """Per-phase step time without events between kernels.
+
+    The combine phase alone: a CUDA graph holding only the step's combine
+    launch, replayed `steps` times between two events (its input, the expert
+    outputs, is larger than L2, so back-to-back replays read HBM like the step
+    does).  The dispatch phase (layout + dispatch) is the rest of the clean
+    step: ms_per_step minus that.  Timing the dispatch phase the same way would
+    flatter it, because its input x (56 MiB at the prefill shape) stays in L2
+    between back-to-back replays, while in the step the combine evicts it."""
+    import torch
+
+    if step.fused_decode or step.layout_dispatch:
+        call = lambda: step.cgl.combine(step.y, step.lay.dst_pos, step.w, out=step.out, status=step.status)
+    elif step.dedup:
+        call = lambda: step.cgl.combine(step.y, step.rlay.rank_dst, step.w_rank, out=step.out, status=step.status)
+    else:
+        call = lambda: step.cgl.combine(step.y, step.lay.dst_pos, step.w, out=step.out, status=step.status)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            call()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / steps
+
+
 def _twin(step: GpuStep) -> GpuStep:
     """A second set of device buffers for the same step (inputs, workspace,
     outputs); the host copies fill its inputs, so only derived inputs are cloned."""
@@ -581,7 +622,8 @@ def base_line(args, wl, n_gpus):
     return {
         "metric": METRIC, "unit": "GB/s", "n_gpus": n_gpus, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
+        "dtype": ("f32 arithmetic; bf16 x in, e4m3 + f32 scale rows out, bf16 combine" if wl.fp8
+                  else "f32 arithmetic; bf16 rows"), "data": "synthetic",
         "config": {
             "workload": workload_label(wl, getattr(args, "dedup", False)), "num_tokens": wl.num_tokens, "hidden": wl.hidden,
             "num_experts": wl.num_experts, "num_groups": wl.num_groups, "topk_group": wl.topk_group,
@@ -695,8 +737,9 @@ def run_ours(args):
             per_phase[i] += ev[i].elapsed_time(ev[i + 1])
     per_phase = [v / args.steps for v in per_phase]
     ms_instr = evs[0][0].elapsed_time(evs[-1][-1]) / args.steps
-    red = max_over_ranks([ms, ms_instr] + per_phase, device=dev)
-    ms, ms_instr, per_phase = red[0], red[1], red[2:]
+    ms_comb = time_phase_graphs(step, args.steps) if not step.wl.with_grad else None
+    red = max_over_ranks([ms, ms_instr, ms_comb or 0.0] + per_phase, device=dev)
+    ms, ms_instr, ms_comb, per_phase = red[0], red[1], (red[2] if ms_comb is not None else None), red[3:]
     status_bits = step.cgl.status_bits(step.status)
 
     e2e = None
@@ -727,11 +770,8 @@ def run_ours(args):
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
             "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
             "bytes_per_launch": kernels[dom]["bytes"],
-            "achieved_alone": alone[dom]["gbs"] if dom in alone else None,
-            "frac_alone": alone[dom]["frac_of_peak"] if dom in alone else None,
-            "timing": ("achieved / frac: CUDA events around each launch in the instrumented pass (launch gap "
-                       "included); achieved_alone / frac_alone: the same kernel launched back to back "
-                       "(kernels_alone)")}
+            "timing": ("in the step: CUDA events on the launching stream around each launch of the kernel over "
+                       "the K steps of the instrumented pass (the gap the events add included)")}
     line = base_line(args, wl, world)
     value = step.step_bytes() * world / (ms * 1e-3) / 1e9
     line.update({
@@ -739,7 +779,7 @@ def run_ours(args):
         "kernels_alone": alone,
         "kernels_alone_timing": ("each kernel of the step alone: a CUDA graph of 20 back-to-back launches replayed "
                                  "to about min(K, 200) launches between two CUDA events, after 3 warm-up launches"),
-        "dispatch_plus_combine_us": sum(kernels[n]["us"] for n in kernels if n != "layout"),
+
         "gpu_launches": args.steps * sum(p[1] for p in phases),
         "launch": "eager" if args.no_graph else "CUDA graph of one step, replayed K times (e2e and per-kernel passes eager)",
         "kernel_timing": ("per-kernel us from a second pass of the same K steps with a CUDA event "
@@ -747,6 +787,18 @@ def run_ours(args):
                           "each includes the launch gap the events add"),
         "clocks": clocks, "device_status": status_bits or "ok",
     })
+    if ms_comb is not None:
+        nb = {n: b for n, _, b in phases}
+        comb_b = nb.get("combine", 0)
+        line.update({
+            "dispatch_us": (ms - ms_comb) * 1e3, "combine_us": ms_comb * 1e3,
+            "dispatch_gbs": (step.step_bytes() - comb_b) / ((ms - ms_comb) * 1e-3) / 1e9,
+            "combine_gbs": comb_b / (ms_comb * 1e-3) / 1e9,
+            "phase_timing": ("no event between kernels: combine_us = a CUDA graph of the step's combine launch "
+                             "alone, replayed K times (its expert-output input exceeds L2); dispatch_us = "
+                             "ms_per_step - combine_us (layout and dispatch, with the transitions of the step); "
+                             "the instrumented per-kernel split is under 'kernels'"),
+        })
     if e2e:
         line["e2e"] = e2e
     if not args.no_cpu_baseline and world == 1 and not args.dedup:

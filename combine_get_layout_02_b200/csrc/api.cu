@@ -324,11 +324,10 @@ cgl_status cgl_layout_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
                                       static_cast<cudaStream_t>(stream));
 }
 
-cgl_status cgl_selftest_bounded_wait(const uint64_t *flags, int nflags, uint32_t *status_dev,
-                                     void *stream) {
-    if (!flags || !status_dev || nflags < 1 || nflags > 4096) return CGL_EINVAL;
-    if (!aligned(flags, 8) || !aligned(status_dev, 4)) return CGL_EALIGN;
-    return launch_wait_probe(flags, nflags, status_dev, static_cast<cudaStream_t>(stream));
+cgl_status cgl_selftest_bounded_wait(uint64_t *workspace, int nflags, uint32_t *status_dev, void *stream) {
+    if (!workspace || !status_dev || nflags < 1 || nflags > 4096) return CGL_EINVAL;
+    if (!aligned(workspace, 8) || !aligned(status_dev, 4)) return CGL_EALIGN;
+    return launch_wait_probe(workspace, nflags, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -75,8 +75,9 @@ cgl_status launch_combine(const uint16_t *y, int64_t recv_rows, const int32_t *d
                           const float *w, int64_t n, int h, int k, uint16_t *out, int num_sms,
                           uint32_t *status, cudaStream_t stream);
 
-// One block running the layout's bounded inter-block wait on flags no kernel sets.
-cgl_status launch_wait_probe(const uint64_t *flags, int nflags, uint32_t *status, cudaStream_t stream);
+// One block running the layout's bounded inter-block wait, with its exit path
+// (generation advance), on a workspace header whose flags hold no tag it waits for.
+cgl_status launch_wait_probe(uint64_t *ws, int nflags, uint32_t *status, cudaStream_t stream);
 
 // Dynamic shared memory of the fused decode kernel (bytes).
 size_t decode_fused_smem_bytes(int64_t n, int k, int E, int R);

@@ -3,7 +3,8 @@
 //
 // The DeepEP pages describe dispatch only as routing each token to its gated
 // experts, with the host waiting on GPU-made receive counts (brainleap "Day2
-// DeepEP", caption "CPU 将隐式地等待 GPU 接收到的计数信号").  The order inside
+// DeepEP", section "All-to-All通信", the figure caption on the host waiting for
+// the receive counts).  The order inside
 // an expert is ascending token order: the result equals one sequential walk
 // over t = 0..N-1, j = 0..k-1 that hands out the next free row of each expert.
 //
@@ -52,10 +53,18 @@
 // fence follows (an acquire load per poll would invalidate L1 every time).
 // One exchange round only: on this part each dependent round trip through L2
 // costs about a microsecond, more than the column sums it would save.  The
-// tag is a generation counter kept in the workspace (+1 per launch), so it
-// changes on every launch, replays of a captured graph included.  Otherwise two kernels run (counts, then bases +
+// tag's low half is a generation counter kept in the workspace, its high half
+// a per-call value from the host with the top bit set (so no count word and no
+// zeroed word ever equals a tag).  Every launch advances the generation by
+// exactly one compare-and-swap from the value its blocks read, on success (block
+// 0, after its wait) and on a timeout (every block that gave up), so no two
+// launches on one workspace share a tag: not graph replays (same host value,
+// new generation), and not a launch after one that timed out, whose published
+// flags would otherwise match the next launch's tag before that launch's blocks
+// had written their counts.  Otherwise two kernels run (counts, then bases +
 // rows), the second with programmatic dependent launch; it recomputes the
 // cheap in-warp ranks.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -128,11 +137,12 @@ __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// The tag of a launch: the host's per-call salt (top bit set) in the high
+// half, generation g0 + 1 in the low half.  Counts (non-negative int32 or
+// 16-bit pairs) never have the top bit of a high half set.
+__device__ __forceinline__ uint64_t launch_tag(uint32_t salt, uint64_t g0) {
+    return ((uint64_t)salt << 32) | ((g0 + 1) & 0xFFFFFFFFull);
 }
-// Flags hold this constant in their high half; counts (non-negative int32) never do.
-constexpr uint64_t kTagHigh = 0x9E3779B9ull << 32;
 
 
 // Barrier of the 256 layout threads (warps 0-7, hardware barrier 1).  In the
@@ -713,10 +723,17 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
 // loads (one L2 read each, no L1 invalidation, all in flight together) until
 // every lane has seen its flags; then a gpu-scope fence makes the other
 // blocks' earlier writes visible, and the block barrier hands that on to the
-// whole block.  Returns true for the whole
-// block when every flag was seen; otherwise reports CGL_ETIMEOUT and returns
-// false for the whole block.  All threads of the block must call it.
-__device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint32_t *status) {
+// whole block.  On the way out the launch's generation advances from g0 (the
+// value this block read at its start) to g0 + 1 by compare-and-swap: block 0
+// does it after a successful wait (every block has read the generation by
+// then, since every flag is published), and every block that gave up does it
+// too, so a timed-out launch also leaves the next launch a new tag.  The first
+// swap wins; later ones find the word changed and do nothing.  Returns true
+// for the whole block when every flag was seen; otherwise reports
+// CGL_ETIMEOUT and returns false for the whole block.  All threads of the
+// block must call it.
+__device__ bool wait_for_flags(uint64_t *gen, uint64_t g0, const uint64_t *flags, int nb, uint64_t tag,
+                               uint32_t *status) {
     bool timed_out = false;
     if (threadIdx.x < 32) {
         const long long start = clock64();
@@ -728,19 +745,26 @@ __device__ bool wait_for_flags(const uint64_t *flags, int nb, uint64_t tag, uint
         }
         __threadfence();
     }
-    if (lsync_or(timed_out)) {
+    const bool failed = lsync_or(timed_out);
+    if (threadIdx.x == 0 && (failed || blockIdx.x == 0))
+        atomicCAS(reinterpret_cast<unsigned long long *>(gen), (unsigned long long)g0,
+                  (unsigned long long)(g0 + 1));
+    if (failed) {
         if (threadIdx.x == 0) report(status, 1u << CGL_ETIMEOUT);
         return false;
     }
     return true;
 }
 
-// Self-test of the bounded wait: one block waits for flags that hold a tag no
-// kernel writes (kTagHigh | 0, generation 0 is never a launch's tag), so it
-// must give up after ~1 s and report CGL_ETIMEOUT.
-__global__ void __launch_bounds__(kThreads) wait_probe_kernel(const uint64_t *flags, int nflags,
-                                                              uint32_t *status) {
-    wait_for_flags(flags, nflags, kTagHigh, status);
+// Self-test of the bounded wait: one block takes `ws` as a layout workspace
+// header (word 0 the generation, then nflags flags) and waits for the tag of
+// salt 0, which no layout launch uses (their salts have the top bit set), so
+// on zeroed or layout-written flags it must give up after ~1 s, report
+// CGL_ETIMEOUT and advance the generation, exactly as a layout block that
+// timed out does.
+__global__ void __launch_bounds__(kThreads) wait_probe_kernel(uint64_t *ws, int nflags, uint32_t *status) {
+    const uint64_t g0 = ld_relaxed_u64(ws);
+    wait_for_flags(ws, g0, ws + 1, nflags, launch_tag(0u, g0), status);
 }
 
 template <int NT = kThreads>
@@ -759,7 +783,7 @@ __device__ void zero_words(int32_t *p, int n) {
 // Returns false (the whole group of 256) when the inter-block wait timed out.
 template <bool kRankKeys, int CH, int U = kColUnroll, bool kU16 = false>
 __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
-                             int key_div, int T, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                             int key_div, int T, uint64_t *flags, uint32_t salt, int32_t *ws_e, int32_t *ws_r,
                              int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                              uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
                              int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
@@ -769,13 +793,14 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     const int nb = gridDim.x, b = blockIdx.x;
     const bool with_ranks = in_rank != nullptr;
 
-    // This launch's tag: generation + 1.  Every block reads the generation before
-    // it publishes its flag, and block 0 advances it only after it has seen every
-    // flag, so all blocks agree and the next launch (a graph replay too) gets a new tag.
+    // This launch's tag: the host's salt and generation + 1.  Every block reads
+    // the generation before it publishes its flag, and it advances only when a
+    // block leaves the wait (wait_for_flags), so all blocks of a launch agree and
+    // the next launch (a graph replay too, or one after a timeout) gets a new tag.
     uint64_t *gen = flags;
     flags += 1;
-    const uint64_t g0 = ld_relaxed_u64(gen) & 0xFFFFFFFFull;
-    const uint64_t tag = kTagHigh | ((g0 + 1) & 0xFFFFFFFFull);
+    const uint64_t g0 = ld_relaxed_u64(gen);
+    const uint64_t tag = launch_tag(salt, g0);
     PairsT<CH> P;
     const bool bad = load_pairs<CH>(idx, n, k, E_ids, b, T, P);   // in flight while zeroing
     zero_words(s.wc, kWarps * E);
@@ -815,8 +840,7 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
 
     // every block's counts must be visible before the bases
-    if (!wait_for_flags(flags, nb, tag, status)) return false;
-    if (b == 0 && tid == 0) st_relaxed_u64(gen, (g0 + 1) & 0xFFFFFFFFull);
+    if (!wait_for_flags(gen, g0, flags, nb, tag, status)) return false;
 
     bases_and_rows<true, kRankKeys, CH, false, kThreads, U, kU16>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
                                                             tokens_per_expert, tokens_per_rank, expert_offset,
@@ -828,7 +852,7 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
 template <bool kRankKeys, int CH>
 __global__ void __launch_bounds__(kThreads)
 layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
-                    int key_div, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                    int key_div, uint64_t *flags, uint32_t salt, int32_t *ws_e, int32_t *ws_r,
                     int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                     uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
                     int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
@@ -836,7 +860,7 @@ layout_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     extern __shared__ __align__(16) int32_t smem_fused[];
     __shared__ int32_t scan_tmp[32];
     const Smem s = carve(0, smem_fused, k, E, R);
-    layout_block<kRankKeys, CH>(idx, n, k, E, R, cap, E_ids, key_div, tokens_per_block(k, CH), flags, ws_e, ws_r,
+    layout_block<kRankKeys, CH>(idx, n, k, E, R, cap, E_ids, key_div, tokens_per_block(k, CH), flags, salt, ws_e, ws_r,
                                 tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
                                 recv_src, recv_rows, status, s, scan_tmp, nullptr);
 }
@@ -1237,7 +1261,7 @@ __device__ void store_fp8_rows(int k, int h, int tl, int cnt, const int32_t *s_d
 template <int CH>
 __global__ void __launch_bounds__(kLdThreads, 1)
 layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int T,
-                           int B, uint64_t *flags, int32_t *ws_e, int32_t *ws_r,
+                           int B, uint64_t *flags, uint32_t salt, int32_t *ws_e, int32_t *ws_r,
                            int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
                            uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
                            int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
@@ -1255,7 +1279,8 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
     const int nt = t0 < n ? (int)(n - t0 < T ? n - t0 : T) : 0;
     const int cnt0 = nt < B ? nt : B;   // == nt: the host launches this kernel only when B >= T
     if (threadIdx.x < kThreads) {
-        const bool ok = layout_block<false, CH, kLdColUnroll, true>(idx, n, k, E, R, cap, E, E / R, T, flags, ws_e, ws_r,
+        const bool ok = layout_block<false, CH, kLdColUnroll, true>(idx, n, k, E, R, cap, E, E / R, T, flags, salt,
+                                                ws_e, ws_r,
                                                 tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
                                                 max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp,
                                                 s_dst);
@@ -1273,6 +1298,15 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
 // ------------------------------------------------------------------ host side
 
 std::mutex g_mu;
+
+// Per-call salt for the exchange tags: a process-wide call counter, spread
+// over 31 bits by an odd multiplier (a bijection), with the top bit set.
+std::atomic<uint32_t> g_calls{0};
+uint32_t next_salt() {
+    const uint32_t c = g_calls.fetch_add(1, std::memory_order_relaxed);
+    return 0x80000000u | ((c * 0x9E3779B1u) & 0x7FFFFFFFu);
+}
+
 int g_fused_ctas_per_sm[2][3][64] = {{{0}}};   // fused-kernel occupancy at kSmemDefault, per mode, CH, device
 
 __host__ __device__ constexpr int ch_slot(int ch) { return ch == 1 ? 0 : (ch == 2 ? 1 : 2); }
@@ -1463,7 +1497,7 @@ cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, in
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t err = cudaLaunchKernelEx(
-        &cfg, layout_dispatch_fp8_kernel<CH>, idx, n, k, E, R, cap, sh.T, sh.B, flags, ws_e, ws_r,
+        &cfg, layout_dispatch_fp8_kernel<CH>, idx, n, k, E, R, cap, sh.T, sh.B, flags, next_salt(), ws_e, ws_r,
         tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src, recv_rows, x, h,
         recv_x, recv_scale, scale_bulk, status);
     if (err == cudaSuccess) return CGL_OK;
@@ -1551,7 +1585,8 @@ cgl_status launch_layout_ch(const int32_t *idx, int64_t n, int k, int E_ids, int
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const cudaError_t err = cudaLaunchKernelEx(
-            &cfg, layout_fused_kernel<kRankKeys, CH>, idx, n, k, E, R, cap, E_ids, key_div, flags, ws_e, ws_r,
+            &cfg, layout_fused_kernel<kRankKeys, CH>, idx, n, k, E, R, cap, E_ids, key_div, flags, next_salt(),
+            ws_e, ws_r,
             tokens_per_key, tokens_per_rank, in_rank, key_offset, max_count, dst_pos, recv_src, recv_rows,
             status);
         if (err == cudaSuccess) return CGL_OK;
@@ -1634,8 +1669,8 @@ cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R
                                     max_count, rank_dst, recv_token, ws, status, stream);
 }
 
-cgl_status launch_wait_probe(const uint64_t *flags, int nflags, uint32_t *status, cudaStream_t stream) {
-    wait_probe_kernel<<<1, kThreads, 0, stream>>>(flags, nflags, status);
+cgl_status launch_wait_probe(uint64_t *ws, int nflags, uint32_t *status, cudaStream_t stream) {
+    wait_probe_kernel<<<1, kThreads, 0, stream>>>(ws, nflags, status);
     return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 

@@ -10,7 +10,8 @@
  *   - "DeepEP ... CPO" GitHub-issue mirror, section "Technical Overview of DeepEP";
  *   - 智东西 news article (yunnanlong.com), the feature list and "具体性能方面";
  *   - brainleap.ai "【Day2】DeepEP", sections "DeepEP是什么", "All-to-All通信"
- *     (combine accumulates) and the caption "CPU 将隐式地等待 GPU 接收到的计数信号";
+ *     (combine accumulates) and that section's figure caption on the host
+ *     waiting for the GPU's receive counts;
  *   - flashmla.org/de "DeepEP", the feature and benchmark-setting paragraphs.
  * Here the expert-parallel ranks are logical partitions of ONE GPU: rank r owns
  * experts [r*E/R, (r+1)*E/R), every "send" is a row copy inside this GPU's
@@ -32,6 +33,15 @@
  *     `status_dev` may be NULL, in which case those errors go unreported (the
  *     kernels still skip the offending copies).  No kernel traps or asserts.
  *   - Calls that share output buffers must not overlap on the GPU.
+ *   - Workspaces take any contents.  The layout's blocks signal one another
+ *     through 64-bit tags in the workspace: a per-call value from the host
+ *     (unique among the process's first 2^31 calls, top bit set) and the
+ *     workspace's launch count, which every launch advances, one that timed out
+ *     included.  So no word that an earlier call of this library left in a
+ *     workspace equals a later call's tag (graph replays of one captured call
+ *     share the host value and differ in the count), and neither does zeroed
+ *     memory or a count word; other data would have to equal the 64-bit tag
+ *     exactly.
  *   - Limits: num_topk in [1, 32]; num_experts in [1, 1024];
  *     num_tokens * num_topk < 2^31; num_experts % num_ranks == 0.
  */
@@ -95,7 +105,8 @@ int cgl_layout_kernel_count(int64_t num_tokens, int num_topk, int num_experts, i
  * logical rank receives, where they start, and the receive row of every
  * (token, slot) copy.  Pages: the dispatch described under "DeepEP是什么" and
  * "All-to-All通信" (brainleap "Day2 DeepEP"), whose receive counts the host
- * waits on (caption "CPU 将隐式地等待 GPU 接收到的计数信号").
+ * waits on (the figure caption in "All-to-All通信" on the host waiting for the
+ * receive counts).
  *
  * In (device):
  *   topk_idx          int32 [num_tokens, num_topk]; expert id per slot, -1 = no copy.
@@ -134,7 +145,8 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t num_tokens, int num_t
  * copy to each logical rank that hosts at least one of its experts, instead of
  * one copy per expert.  Pages: the normal kernels' per-destination transfers
  * and their receive counts ("All-to-All通信", the dispatch bullet: send,
- * forward, receive per destination; caption "CPU 将隐式地等待 GPU 接收到的计数信号").
+ * forward, receive per destination; the figure caption there on the host
+ * waiting for the receive counts).
  * Reading: this is the is_token_in_rank view of dispatch; the receiving rank
  * then serves its local experts and returns one partial row per token.
  *
@@ -361,15 +373,18 @@ cgl_status cgl_combine_backward(const uint16_t *grad_out, const uint16_t *y, int
 
 /*
  * cgl_selftest_bounded_wait -- diagnostic for failure detection.  Runs the
- * layout's inter-block wait (the only wait in any kernel of this library) in
- * one block, on `nflags` device words that no kernel writes with the tag it
- * waits for.  The wait must give up after ~1 s (2^31 SM cycles), OR
- * 1u << CGL_ETIMEOUT into *status_dev and return; the stream and the context
- * stay usable.  flags: device, 8-byte aligned, nflags in [1, 4096], any
- * contents (zeroed memory works).  The pages have no counterpart.
+ * layout's inter-block wait (the only software wait in any kernel of this
+ * library) in one block, exit path included, on a layout workspace header:
+ * workspace[0] is the generation word and workspace[1 .. nflags] are the flags.
+ * It waits for a tag that no layout launch writes, so on zeroed memory, or on
+ * a header that layout calls have used, it must give up after ~1 s (2^31 SM
+ * cycles), OR 1u << CGL_ETIMEOUT into *status_dev, advance the generation word
+ * by one (as a layout block that times out does, so that the next layout call
+ * on that workspace gets a new tag) and return; the stream and the context
+ * stay usable.  workspace: device, 8-byte aligned, 1 + nflags words;
+ * nflags in [1, 4096].  The pages have no counterpart.
  */
-cgl_status cgl_selftest_bounded_wait(const uint64_t *flags, int nflags, uint32_t *status_dev,
-                                     void *stream);
+cgl_status cgl_selftest_bounded_wait(uint64_t *workspace, int nflags, uint32_t *status_dev, void *stream);
 
 #ifdef __cplusplus
 }

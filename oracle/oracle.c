@@ -11,7 +11,8 @@
  *     "Technical Overview"; brainleap "Day2 DeepEP", "DeepEP是什么" and the
  *     combine paragraph of "All-to-All通信");
  *   - FP8 dispatch, BF16 combine (same pages, benchmark settings);
- *   - the host reads a GPU-made receive count ("CPU 将隐式地等待 GPU 接收到的计数信号").
+ *   - the host reads a GPU-made receive count (brainleap "Day2 DeepEP", section
+ *     "All-to-All通信", the figure caption on the host waiting for receive counts).
  * Everything finer (1x128 scale blocks, amax/448 scales, RNE + saturation,
  * ascending-token stable order, fixed-order fp32 combine) is this library's
  * reading of the benchmark spec; each function states the reading it takes.

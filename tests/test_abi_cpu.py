@@ -180,3 +180,36 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(cgl, "LIB_PATH", str(tmp_path / "libcgl.so"))
     with pytest.raises(RuntimeError, match="not built"):
         cgl.layout_workspace_bytes(4096, 8, 256, 64)
+
+
+def test_noalloc_limits_at_their_exact_boundaries(L):
+    """cgl_get_layout_noalloc refuses exactly the sizes past its two limits.
+
+    A refused size returns CGL_EINVAL before anything else.  An accepted size
+    goes on to the scratch lookup (CGL_ECUDA without a device) or, where a
+    device exists, to cgl_get_layout's checks, which refuse the misaligned
+    is_token_in_rank passed here (CGL_EALIGN): nothing is launched either way."""
+    f = L.cgl_get_layout_noalloc
+    P, I64, I = C.c_void_p, C.c_int64, C.c_int
+    f.argtypes = [P, I64, I, I, I, C.POINTER(cgl.Opts), P, P, P, P, P, P, P, P, P]
+    f.restype = I
+    p = FAKE
+
+    def call(n, k, E, R):
+        return f(p, n, k, E, R, None, p, p, p + 2, p, p, p, p, p, None)
+
+    accepted = (cgl.ECUDA, cgl.EALIGN)
+    # scratch: 512 KiB holds the per-block counts of exactly 52,096 tokens at top-8, E=256, R=64
+    assert L.cgl_layout_workspace_bytes(52096, 8, 256, 64) == 512 * 1024
+    assert L.cgl_layout_workspace_bytes(52097, 8, 256, 64) > 512 * 1024
+    assert call(52096, 8, 256, 64) in accepted
+    assert call(52097, 8, 256, 64) == cgl.EINVAL
+    # shared memory: 12 E + R + T ceil(R / 32) <= 9984 with T = min(256, 1024 / k)
+    # (R = 1, k = 1: T = 256, so E <= 810; R = 64: E <= 784, the next multiple of 64 is 832)
+    assert call(1000, 1, 810, 1) in accepted
+    assert call(1000, 1, 811, 1) == cgl.EINVAL
+    assert call(1000, 1, 768, 64) in accepted
+    assert call(1000, 1, 832, 64) == cgl.EINVAL
+    # k = 8, R = 32: T = 128 tokens per block, 12 E + 32 + 128 <= 9984 -> E <= 818 (800 and 832 are multiples of 32)
+    assert call(1000, 8, 800, 32) in accepted
+    assert call(1000, 8, 832, 32) == cgl.EINVAL

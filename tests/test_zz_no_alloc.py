@@ -4,11 +4,12 @@ This entry point is for callers that cannot allocate device memory (hosts that
 pass only pre-planned input/output buffers, callers that must avoid the
 synchronisation of cudaFree, C-only callers without a CUDA allocator); its
 scratch is a fixed device array inside libcgl.so, shared by all calls.  The
-test runs two calls in a row on different inputs, so that the second sees
-whatever the first left in that array, and compares each with cgl_get_layout
-(the existing entry point, with a caller-allocated workspace) bit for bit, the
-tolerance for integer outputs.  It also checks that sizes past the array's
-limit are refused before any launch.  The file sorts last so that a run that
+test runs several calls in a row on different inputs and shapes, so that each
+sees whatever the one before left in that array, and compares each with
+cgl_get_layout (the existing entry point, with a caller-allocated workspace)
+bit for bit, the
+tolerance for integer outputs, and with the CPU oracle.  It also checks that
+sizes past the array's limit are refused before any launch.  The file sorts last so that a run that
 stops at the first failure has already run everything else.
 """
 
@@ -63,23 +64,51 @@ def _reference(idx: torch.Tensor, E: int, R: int, cap: int = 0):
     return {f: getattr(lay, f) for f in FIELDS}, st
 
 
-def test_noalloc_matches_get_layout_on_two_calls_in_a_row():
+def _oracle_check(oracle_mod, got, idx_np, E, R, cap):
+    L = oracle_mod.get_layout(idx_np, E, R, cap)
+    for f in FIELDS:
+        if f == "max_count":
+            assert int(got[f].item()) == L.max_count
+            continue
+        g, r = got[f].cpu().numpy(), getattr(L, f)
+        assert g.shape == r.shape and np.array_equal(g, r), f
+    return L
+
+
+def test_noalloc_matches_oracle_and_get_layout_on_calls_in_a_row(oracle_mod):
+    """Consecutive calls of different shapes share the scratch array: each later
+    call runs on what the one before left in it (generation word, flags and count
+    rows of another block count, E and R).  Every call takes the path that
+    exchanges counts through the array (several layout blocks), except the
+    padded decode call, which needs none.  Each output is compared bit for bit
+    with the oracle and with cgl_get_layout."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    cases = []
-    a = W.make_inputs("skewed", 0)          # 16384 tokens: the larger scratch footprint first
-    cases.append((torch.from_numpy(a.topk_idx).to(dev), 256, 64, 0))
-    b = W.make_inputs("decode", 0)          # then a small padded layout over the leftovers
-    idx_b = torch.from_numpy(b.topk_idx).to(dev)
-    cap = int(_reference(idx_b, 256, 32)[0]["max_count"].item())
-    cases.append((idx_b, 256, 32, cap))
-    for idx, E, R, c in cases:
+    pre = W.make_inputs("prefill", 0)           # 64 blocks of 64 tokens, E=256, R=64
+    skw = W.make_inputs("skewed", 0)            # 128 blocks of 128 tokens, E=256, R=32 (ranks of 8 experts)
+    dec = W.make_inputs("decode", 0)
+    cap_pre = oracle_mod.get_layout(pre.topk_idx, 256, 64).max_count
+    cap_dec = oracle_mod.get_layout(dec.topk_idx, 256, 32).max_count
+    cases = [
+        (pre.topk_idx, 256, 64, 0),
+        (skw.topk_idx, 256, 32, 0),
+        (pre.topk_idx, 256, 64, cap_pre - 3),   # padded, some experts overflow (CGL_ECAPACITY)
+        (dec.topk_idx, 256, 32, cap_dec),
+        (pre.topk_idx[:1500], 256, 64, 0),      # 47 blocks of 32 tokens
+        (pre.topk_idx, 256, 64, 0),
+    ]
+    for idx_np, E, R, c in cases:
+        idx = torch.from_numpy(np.ascontiguousarray(idx_np)).to(dev)
         got, st = _noalloc(idx, E, R, c)
         ref, st_ref = _reference(idx, E, R, c)
         torch.cuda.synchronize()
+        L = _oracle_check(oracle_mod, got, idx_np, E, R, c)
         for f in FIELDS:
             assert torch.equal(got[f], ref[f]), f
-        assert int(st.item()) == int(st_ref.item()) == 0
+        bits = int(st.item())
+        assert bits == int(st_ref.item())
+        assert bool(bits & (1 << cgl.ECAPACITY)) == bool(L.flags & oracle_mod.FLAG_CAPACITY)
+        assert not bits & ~(1 << cgl.ECAPACITY)
 
 
 def test_noalloc_refuses_sizes_past_its_scratch():
