@@ -29,6 +29,16 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
     return r;
 }
 
+// 16-byte global load through the non-coherent path, allocated in L1: for
+// reads whose other half of the 32-byte sector the next instruction reads.
+__device__ __forceinline__ uint4 ld_nc_l1_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 // 16-byte global store with the streaming (evict-first) cache hint.
 __device__ __forceinline__ void st_cs_v4(void *p, uint4 v) {
     asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
@@ -83,17 +93,32 @@ __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Ask the TMA engine to bring `bytes` of global memory at `src` into L2 (no
+// data lands in the SM; completion is not tracked).  src 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Widen the low / high BF16 of a 32-bit word to float (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Largest |value| among the 16 BF16 values in (a, b).
+// Largest |value| among the 16 BF16 values in (a, b), as a float (exact: a
+// maximum does not round).  The sign bits are cleared and the maximum taken on
+// BF16 pairs (max.bf16x2), then between the two halves; NaN inputs are outside
+// the contract (the pairwise maximum, like fmaxf, prefers the number).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t p, uint32_t q) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(q));
+    return r;
+}
 __device__ __forceinline__ float absmax16(const uint4 a, const uint4 b) {
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    return m;
+    constexpr uint32_t kAbs = 0x7FFF7FFFu;
+    const uint32_t m01 = bf16x2_max(a.x & kAbs, a.y & kAbs), m23 = bf16x2_max(a.z & kAbs, a.w & kAbs);
+    const uint32_t m45 = bf16x2_max(b.x & kAbs, b.y & kAbs), m67 = bf16x2_max(b.z & kAbs, b.w & kAbs);
+    const uint32_t m = bf16x2_max(bf16x2_max(m01, m23), bf16x2_max(m45, m67));
+    return fmaxf(bf16_lo(m), bf16_hi(m));
 }
 
 // E4M3 codes of the 16 BF16 values in (a, b), each multiplied by inv first.

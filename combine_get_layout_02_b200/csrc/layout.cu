@@ -138,8 +138,8 @@ __device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
     return v;
 }
 // The tag of a launch: the host's per-call salt (top bit set) in the high
-// half, generation g0 + 1 in the low half.  Counts (non-negative int32 or
-// 16-bit pairs) never have the top bit of a high half set.
+// half, generation g0 + 1 in the low half.  Count words (non-negative int32)
+// never have the top bit of a high half set.
 __device__ __forceinline__ uint64_t launch_tag(uint32_t salt, uint64_t g0) {
     return ((uint64_t)salt << 32) | ((g0 + 1) & 0xFFFFFFFFull);
 }
@@ -156,6 +156,13 @@ __device__ __forceinline__ bool lsync_or(bool v) {
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r) : "r"((int)v) : "memory");
     return r != 0;
+}
+
+// Shared-memory add without a return value (red.shared): the pointer must point
+// into shared memory; spelling out the state space keeps the compiler from a
+// generic atomic, which is several times slower here.
+__device__ __forceinline__ void red_shared_add(int32_t *p, int v) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v) : "memory");
 }
 
 // q = e / d for 0 <= e < 1024 and 1 <= d <= 1024 as (e * m) >> 20 with
@@ -494,77 +501,6 @@ __device__ void column_sums(const int32_t *t, int nb, int ncols, int upto, int32
     lsync();
 }
 
-// The same over a table of 16-bit counts (a block's count per key is at most
-// its 1024 pairs), ncols a multiple of 8: one 16-byte load carries 8 columns,
-// so the all-blocks read moves half the bytes of the 32-bit table.
-template <bool kCoherent>
-__device__ __forceinline__ uint4 ld_col8_u16(const uint16_t *p) {
-    const uint4 *q = reinterpret_cast<const uint4 *>(p);
-    return kCoherent ? __ldcg(q) : __ldg(q);
-}
-
-template <bool kCoherent, int U = kColUnroll>
-__device__ void column_sums_u16(const uint16_t *t, int nb, int ncols, int upto, int32_t *out_tot,
-                                int32_t *out_pre, int32_t *part) {
-    const int tid = threadIdx.x;
-    const int nq = ncols / 8;                        // 16-byte loads per row
-    int G = nq >= kThreads ? 1 : kThreads / nq;
-    if (2 * G * ncols > kPartWords) G = kPartWords / (2 * ncols);
-    if (G < 1) G = 1;
-    const int q0 = G > 1 ? tid % nq : tid;
-    const int g = G > 1 ? tid / nq : 0;
-    const int qstep = G > 1 ? nq : kThreads;
-    if (g < G) {
-        for (int q = q0; q < nq; q += qstep) {
-            int32_t tot[8] = {0, 0, 0, 0, 0, 0, 0, 0}, pre[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            for (int r0 = g; r0 < nb; r0 += G * U) {
-                uint4 v[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int r = r0 + u * G;
-                    v[u] = r < nb ? ld_col8_u16<kCoherent>(t + (int64_t)r * ncols + q * 8) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int32_t below = r0 + u * G < upto ? 1 : 0;
-                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int32_t lo = (int32_t)(w[i] & 0xFFFFu), hi = (int32_t)(w[i] >> 16);
-                        tot[2 * i] += lo;
-                        tot[2 * i + 1] += hi;
-                        pre[2 * i] += below * lo;
-                        pre[2 * i + 1] += below * hi;
-                    }
-                }
-            }
-            for (int c = 0; c < 8; ++c) {
-                const int col = q * 8 + c;
-                if (G > 1) {
-                    part[g * ncols + col] = tot[c];
-                    part[(G + g) * ncols + col] = pre[c];
-                } else {
-                    out_tot[col] = tot[c];
-                    if (out_pre) out_pre[col] = pre[c];
-                }
-            }
-        }
-    }
-    if (G > 1) {
-        lsync();
-        for (int col = tid; col < ncols; col += kThreads) {
-            int32_t a = 0, b = 0;
-            for (int gg = 0; gg < G; ++gg) {
-                a += part[gg * ncols + col];
-                b += part[(G + gg) * ncols + col];
-            }
-            out_tot[col] = a;
-            if (out_pre) out_pre[col] = b;
-        }
-    }
-    lsync();
-}
-
 // Exclusive scan of v[0..n) in shared memory (n <= kMaxExperts) into out[];
 // returns the total.  All threads of the block must call it.
 template <int NT = kThreads>
@@ -605,7 +541,7 @@ __device__ int32_t block_exclusive_scan(const int32_t *v, int32_t *out, int n, i
 // Bases, the global outputs (block 0) and the rows of the block's pairs.
 // kTotalsGiven: s.total / s.base (copies in earlier blocks) are already set.
 template <bool kCoherent, bool kRankKeys, int CH = kChunks, bool kTotalsGiven = false, int NT = kThreads,
-          int U = kColUnroll, bool kU16 = false>
+          int U = kColUnroll>
 __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t n, int k, int E, int R,
                                int cap, int64_t recv_rows, int32_t *__restrict__ tokens_per_expert,
                                int32_t *__restrict__ tokens_per_rank, int32_t *__restrict__ expert_offset,
@@ -637,11 +573,7 @@ __device__ void bases_and_rows(const int32_t *ws_e, const int32_t *ws_r, int64_t
         }
         lsync();
     } else {
-        if constexpr (kU16)
-            column_sums_u16<kCoherent, U>(reinterpret_cast<const uint16_t *>(ws_e), nb, E, b, s.total, s.base,
-                                          s.part);
-        else
-            column_sums<kCoherent, U>(ws_e, nb, E, b, s.total, s.base, s.part);
+        column_sums<kCoherent, U>(ws_e, nb, E, b, s.total, s.base, s.part);
     }
     if (rank_sums) {
         for (int r = rcol; r < R; r += nb * (NT / 32)) {   // warp-uniform
@@ -781,7 +713,7 @@ __device__ void zero_words(int32_t *p, int n) {
 // for the key transform; in_rank == nullptr skips the rank sets (rank mode).
 // s_dst (optional, shared memory, T k words) also receives the block's rows.
 // Returns false (the whole group of 256) when the inter-block wait timed out.
-template <bool kRankKeys, int CH, int U = kColUnroll, bool kU16 = false>
+template <bool kRankKeys, int CH, int U = kColUnroll>
 __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int E_ids,
                              int key_div, int T, uint64_t *flags, uint32_t salt, int32_t *ws_e, int32_t *ws_r,
                              int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
@@ -816,18 +748,13 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     if (nb == 1) {   // nothing to exchange
         if (with_ranks) write_rank_rows<CH>(R, in_rank, s, P);
         if (lsync_or(bad) && tid == 0) report(status, kErrRange);
-        bases_and_rows<true, kRankKeys, CH, false, kThreads, U, kU16>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+        bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
                                                                 tokens_per_expert, tokens_per_rank, expert_offset,
                                                                 max_count, dst_pos, recv_src, status, s, P,
                                                                 scan_tmp, s_dst);
         return true;
     }
-    if constexpr (kU16) {   // 16-bit count rows (E % 8 == 0; counts <= 1024)
-        uint16_t *row = reinterpret_cast<uint16_t *>(ws_e) + (int64_t)b * E;
-        for (int i = tid; i < E; i += kThreads) row[i] = (uint16_t)s.he[i];
-    } else {
-        for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
-    }
+    for (int i = tid; i < E; i += kThreads) ws_e[(int64_t)b * E + i] = s.he[i];
     for (int i = tid; i < R; i += kThreads) ws_r[(int64_t)b * R + i] = s.hr[i];
     const bool any_bad = lsync_or(bad);   // also orders the workspace writes before the flag
     if (tid == 0) {
@@ -842,7 +769,7 @@ __device__ bool layout_block(const int32_t *__restrict__ idx, int64_t n, int k, 
     // every block's counts must be visible before the bases
     if (!wait_for_flags(gen, g0, flags, nb, tag, status)) return false;
 
-    bases_and_rows<true, kRankKeys, CH, false, kThreads, U, kU16>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
+    bases_and_rows<true, kRankKeys, CH, false, kThreads, U>(ws_e, ws_r, n, k, E, R, cap, recv_rows,
                                                             tokens_per_expert, tokens_per_rank, expert_offset,
                                                             max_count, dst_pos, recv_src, status, s, P, scan_tmp,
                                                             s_dst);
@@ -1010,13 +937,240 @@ layout_cluster_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, 
     cluster_wait_acquire();     // the peers have finished reading this CTA's shared memory
 }
 
+// ------------------------------------------------- replicated-count layout
+//
+// Batches up to a few thousand tokens: no exchange between blocks at all.
+// Block b of G owns tokens [b T, b T + T) as above, and learns the global
+// counts by reading every id of the batch itself (N k ids, from L2 after the
+// first block has read them: 128 KiB at 4096 tokens, top-8) into two
+// shared-memory histograms with shared atomics, one per id: copies in tokens
+// before its own (before[e]) and the rest (rest[e]).  total = before + rest
+// gives the expert offsets by one scan over E; a copy's row is expert base +
+// before[e] + the block's own in-order rank (warp offsets + in-warp rank, as
+// above).  The same pass counts distinct tokens for the block's designated
+// ranks r = b, b + G, ... (at most 32 of them; one ballot per rank per 32
+// tokens).  The redundant reads cost every block the same ~N k atomics, which
+// is why it is kept to small and medium batches; in exchange nothing waits on
+// another block, so no cooperative launch, no workspace and no bounded wait.
+
+// Measured on B200 (graph of 20 back-to-back layouts, E = 256, R = 64, top-8):
+// 128 / 1024 / 2048 / 4096 tokens take 5.6 / 7.3 / 8.0 / 10.4 us this way
+// against 6.2 / 8.8 / 9.5 / 10.2 us with the exchange; at 6144 tokens the
+// blocks no longer fit on the GPU at once and it loses (18.9 against 12.1).
+#ifndef CGL_REP_MAX_PAIRS
+#define CGL_REP_MAX_PAIRS 32768
+#endif
+constexpr int64_t kRepMaxPairs = CGL_REP_MAX_PAIRS;   // (token, slot) pairs of the batch
+constexpr int64_t kRepWidePairs = 4096;   // above this, standalone blocks scan with kRepThreads threads
+
+// Shared memory of a replicated-count layout block with T tokens (words):
+// warp counts [8][E], block counts [E], rank sets [T][mask_words(R)], own
+// rank counts [R], total (rest) [E], before / base [E], offsets [E], and 32
+// designated-rank counts.
+__host__ __device__ __forceinline__ size_t rep_smem_words(int T, int E, int R) {
+    return (size_t)kWarps * E + E + (size_t)T * mask_words(R) + R + 3 * (size_t)E + 32;
+}
+
+__device__ Smem carve_rep(int32_t *p, int T, int E, int R) {
+    Smem s = {};
+    s.wc = p; p += kWarps * E;
+    s.he = p; p += E;
+    s.mask = reinterpret_cast<uint32_t *>(p); p += T * mask_words(R);
+    s.hr = p; p += R;
+    s.total = p; p += E;
+    s.base = p; p += E;
+    s.off = p; p += E;
+    s.part = p;   // 32 designated-rank counts
+    return s;
+}
+
+// Designated ranks of block b of G: b + i G for i < rep_designated(b, G, R).
+__host__ __device__ __forceinline__ int rep_designated(int b, int G, int R) {
+    return b < R ? (R - 1 - b) / G + 1 : 0;
+}
+
+// Every id of the batch into before[] (tokens < t0) / rest[] (tokens >= t0),
+// and distinct tokens of the designated ranks b + i G (i < nd <= 32) into
+// dcnt[i].  Warp-uniform loop over groups of 32 tokens, one token per lane;
+// the ids of U groups are loaded before any of them is counted.  KM >= k ids
+// per token are held in registers; kVec: k % 4 == 0 and idx 16-byte aligned
+// (int4 loads).  All 256 layout threads call it.
+template <bool kVec, int KM, int NT>
+__device__ void rep_scan_ids(const int32_t *__restrict__ idx, int64_t n, int k, int E, int64_t t0,
+                             int32_t *before, int32_t *rest, uint32_t rank_magic, int b, int G, int nd,
+                             int32_t *dcnt) {
+    constexpr int U = KM <= 8 ? 2 : 1;   // token groups in flight per warp
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t gmag = div_magic(G);
+    int32_t dc = 0;   // lane i < nd: this warp's count for designated rank i
+    for (int64_t g0 = (int64_t)warp * 32; g0 < n; g0 += (int64_t)NT * U) {
+        int32_t ids[U][KM];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t t = g0 + (int64_t)u * NT + lane;
+            const int32_t *src = idx + t * k;
+            if (kVec) {
+#pragma unroll
+                for (int q = 0; q < KM / 4; ++q) {
+                    int4 v = make_int4(-1, -1, -1, -1);
+                    if (t < n && q * 4 < k) v = __ldg(reinterpret_cast<const int4 *>(src) + q);
+                    ids[u][4 * q] = v.x; ids[u][4 * q + 1] = v.y; ids[u][4 * q + 2] = v.z; ids[u][4 * q + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < KM; ++j) ids[u][j] = (t < n && j < k) ? __ldg(src + j) : -1;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t t = g0 + (int64_t)u * NT + lane;
+            int32_t *cnt = t < t0 ? before : rest;
+            uint32_t hits = 0;
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                const int32_t e = ids[u][j];
+                if (j < k && (uint32_t)e < (uint32_t)E) {
+                    red_shared_add(cnt + e, 1);
+                    const int d = div_small(e, rank_magic) - b;
+                    if (d >= 0) {
+                        const int q = div_small(d, gmag);
+                        if (q * G == d && q < nd) hits |= 1u << q;
+                    }
+                }
+            }
+            if (g0 + (int64_t)u * NT < n) {   // warp-uniform
+                for (int i = 0; i < nd; ++i) {
+                    const int c = __popc(__ballot_sync(0xFFFFFFFFu, (hits >> i) & 1u));
+                    if (lane == i) dc += c;
+                }
+            }
+        }
+    }
+    if (lane < nd && dc) red_shared_add(dcnt + lane, dc);
+}
+
+// The scan over every id by NT threads (all of them must call it).
+template <int NT>
+__device__ void rep_scan(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int64_t t0, bool vec,
+                         const Smem &s) {
+    const int G = gridDim.x, b = blockIdx.x;
+    const int nd = G > 1 ? rep_designated(b, G, R) : 0;
+    const uint32_t rm = div_magic(E / R);
+    if (k <= 8) {
+        if (vec) rep_scan_ids<true, 8, NT>(idx, n, k, E, t0, s.base, s.total, rm, b, G, nd, s.part);
+        else rep_scan_ids<false, 8, NT>(idx, n, k, E, t0, s.base, s.total, rm, b, G, nd, s.part);
+    } else {
+        if (vec) rep_scan_ids<true, kMaxTopk, NT>(idx, n, k, E, t0, s.base, s.total, rm, b, G, nd, s.part);
+        else rep_scan_ids<false, kMaxTopk, NT>(idx, n, k, E, t0, s.base, s.total, rm, b, G, nd, s.part);
+    }
+}
+
+// Zero a replicated-count block's shared counters (NT threads).
+template <int NT>
+__device__ void rep_zero(int T, int E, int R, const Smem &s) {
+    zero_words<NT>(s.wc, kWarps * E);
+    zero_words<NT>(reinterpret_cast<int32_t *>(s.mask), T * mask_words(R));
+    zero_words<NT>(s.hr, R);
+    zero_words<NT>(s.total, E);
+    zero_words<NT>(s.base, E);
+    zero_words<NT>(s.part, 32);
+}
+
+// The block's own part of a replicated-count layout once the scan's counts are
+// in shared memory, run by the 256 threads of warps 0-7 (barrier 1): block b =
+// blockIdx.x of G = gridDim.x owns tokens [b T, b T + T).  Ranks its own copies,
+// writes every layout output of its own tokens, its designated ranks'
+// tokens_per_rank, its share of the recv_src fill, and (block 0) the expert
+// counts, offsets and max; s_dst (optional, shared, T k words) also receives its
+// rows.  P holds the block's ids (load_pairs).  Requires G == 1 or
+// rep_designated(0, G, R) <= 32.
+template <int CH>
+__device__ void rep_finish(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, bool bad,
+                           PairsT<CH> &P, int32_t *__restrict__ tokens_per_expert,
+                           int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
+                           int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
+                           int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
+                           uint32_t *status, const Smem &s, int32_t *scan_tmp, int32_t *s_dst) {
+    const int tid = threadIdx.x;
+    const int G = gridDim.x, b = blockIdx.x;
+    const int nd = G > 1 ? rep_designated(b, G, R) : 0;
+    key_and_rank<false, CH>(idx, k, E, E / R, E, s, P);
+    rank_sets<CH>(k, E, R, s, P);
+    lsync();
+    warp_offsets(E, s);
+    if (G == 1) rank_counts<CH>(k, R, s, P);   // one block: its own tokens are all tokens
+    for (int e = tid; e < E; e += kThreads) s.total[e] += s.base[e];   // rest + before
+    lsync();
+    write_rank_rows<CH>(R, in_rank, s, P);
+    if (G == 1) {
+        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
+    } else if (tid < nd) {
+        tokens_per_rank[b + tid * G] = s.part[tid];
+    }
+    if (lsync_or(bad) && tid == 0) report(status, kErrRange);
+    bases_and_rows<true, false, CH, true>(nullptr, nullptr, n, k, E, R, cap, recv_rows, tokens_per_expert, nullptr,
+                                          expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp,
+                                          s_dst);
+}
+
+// A whole replicated-count layout block run by the 256 threads of warps 0-7.
+template <int CH>
+__device__ void rep_layout_block(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int T,
+                                 bool vec, int32_t *__restrict__ tokens_per_expert,
+                                 int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
+                                 int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
+                                 int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
+                                 uint32_t *status, const Smem &s, int32_t *scan_tmp, int32_t *s_dst) {
+    PairsT<CH> P;
+    const bool bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight while zeroing
+    rep_zero<kThreads>(T, E, R, s);
+    lsync();
+    rep_scan<kThreads>(idx, n, k, E, R, P.t0, vec, s);
+    rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                   max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
+}
+
+// Standalone replicated-count layout: CTAs of NT threads, all of which zero
+// the counters and scan the ids (the scan is latency-bound, so past a few
+// thousand ids it wants every warp the SM can hold: NT = kRepThreads); warps
+// 0-7 then finish the block.
+constexpr int kRepThreads = 1024;
+
+template <int CH, int NT>
+__global__ void __launch_bounds__(NT)
+layout_rep_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int vec,
+                  int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
+                  uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
+                  int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
+                  int32_t *__restrict__ recv_src, int64_t recv_rows, uint32_t *status) {
+    extern __shared__ __align__(16) int32_t smem_rep[];
+    __shared__ int32_t scan_tmp[32];
+    const int T = tokens_per_block(k, CH);
+    const Smem s = carve_rep(smem_rep, T, E, R);
+    griddep_wait();   // the ids, and readers of the outputs, may be the kernels just before
+    PairsT<CH> P;
+    bool bad = false;
+    if (threadIdx.x < kThreads) bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight
+    rep_zero<NT>(T, E, R, s);
+    __syncthreads();
+    rep_scan<NT>(idx, n, k, E, R, (int64_t)blockIdx.x * T, vec != 0, s);
+    __syncthreads();
+    if (threadIdx.x < kThreads)
+        rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                       max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, nullptr);
+}
+
 // Fused decode path: the layout and the FP8 dispatch of a small batch (at most
-// 1024 (token, slot) pairs) in one launch, no workspace.  Every CTA computes the
-// whole layout in shared memory (one layout block's work, so no inter-block
-// exchange), CTA 0 writes the layout outputs, and each CTA then quantises its
-// share of the tokens and writes their copies with 16-byte stores.
+// 1024 (token, slot) pairs) in one launch, no workspace.  CTA b owns tokens
+// [b T, b T + T) (one token per CTA when there are as many SMs as tokens) as a
+// replicated-count layout block: it reads the batch's ids for the global
+// counts, ranks its own copies and keeps their rows in shared memory, then
+// quantises its tokens and writes their copies with 16-byte stores (one
+// thread per 16 values of the CTA's flattened (token, chunk) range; the 8
+// lanes of a 128-value block share one scale).
+template <int CH>
 __global__ void __launch_bounds__(kThreads)
-decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap,
+decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int T, int vec,
                     const uint16_t *__restrict__ x, int h, int32_t *__restrict__ tokens_per_expert,
                     int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
                     int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
@@ -1024,166 +1178,128 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
                     uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, uint32_t *status) {
     extern __shared__ __align__(16) int32_t smem_decode[];
     __shared__ int32_t scan_tmp[32];
-    const Smem s = carve(0, smem_decode, k, E, R);
-    int32_t *s_dst = smem_decode + smem_words(0, k, E, R);   // [n * k] receive row per pair
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool writer = blockIdx.x == 0;
-
+    const Smem s = carve_rep(smem_decode, T, E, R);
+    int32_t *s_dst = smem_decode + rep_smem_words(T, E, R);   // [T k] receive row per own pair
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     griddep_wait();                // ids and x may come from the kernels just before
-    zero_words(s.wc, kWarps * E);
-    zero_words(reinterpret_cast<int32_t *>(s.mask), tokens_per_block(k) * mask_words(R));
-    zero_words(s.hr, R);
+    rep_layout_block<CH>(idx, n, k, E, R, cap, T, vec != 0, tokens_per_expert, tokens_per_rank, in_rank,
+                         expert_offset, max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
     __syncthreads();
-    Pairs P;
-    const bool bad = load_and_rank<false>(idx, n, k, E, E / R, E, 0, tokens_per_block(k), s, P);
-    if (writer) rank_sets(k, E, R, s, P);
-    __syncthreads();
-    warp_offsets(E, s);
-    if (writer) {
-        rank_counts(k, R, s, P);
-        write_rank_rows(R, in_rank, s, P);
-    }
-    __syncthreads();
-    const int32_t m_total = block_exclusive_scan(s.he, s.off, E, scan_tmp);
-    for (int e = tid; e < E; e += kThreads) s.base[e] = cap > 0 ? e * cap : s.off[e];
-    if (writer) {
-        int32_t mx = 0;
-        for (int e = tid; e < E; e += kThreads) {
-            tokens_per_expert[e] = s.he[e];
-            expert_offset[e] = s.off[e];
-            mx = max(mx, s.he[e]);
-        }
-        if (tid == 0) expert_offset[E] = m_total;
-        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        if (lane == 0) scan_tmp[warp] = mx;
-        __syncthreads();
-        if (tid == 0) {
-            int32_t m = 0;
-            for (int w = 0; w < kWarps; ++w) m = max(m, scan_tmp[w]);
-            *max_count = m;
-        }
-        if (cap > 0) {
-            for (int64_t i = tid; i < (int64_t)E * cap; i += kThreads) {
-                const int e = (int)(i / cap);
-                if (i - (int64_t)e * cap >= s.he[e]) recv_src[i] = -1;
-            }
-        } else {
-            for (int64_t i = m_total + tid; i < n * k; i += kThreads) recv_src[i] = -1;
-        }
-        if (__syncthreads_or(bad) && tid == 0) report(status, kErrRange);
-    }
-    __syncthreads();
-    bool over = false;
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int p = pair_of(i);
-        if (p >= P.np) continue;
-        const int32_t e = P.e[i];
-        int32_t d = -1;
-        if (e >= 0) {
-            const int32_t pos = s.base[e] + s.wc[warp * E + e] + P.rk[i];
-            if (cap > 0 && pos - e * cap >= cap) over = true;
-            else if (pos < recv_rows) d = pos;
-        }
-        s_dst[p] = d;
-        if (writer) {
-            dst_pos[p] = d;
-            if (d >= 0) recv_src[d] = p;
-        }
-    }
-    if (writer && over) report(status, kErrCapacity);
-    __syncthreads();
-
-    // dispatch this CTA's tokens: 16 values per thread per pass, 8 lanes per scale block
+    const int64_t t0 = (int64_t)blockIdx.x * T;
+    const int nt = t0 < n ? (int)(n - t0 < T ? n - t0 : T) : 0;
     const int chunks = h >> 4, nblk = h >> 7;
-    for (int64_t t = blockIdx.x; t < n; t += gridDim.x) {
-        for (int c0 = warp * 32; c0 < chunks; c0 += kThreads) {   // warp-uniform
-            const int c = c0 + lane;
-            const bool active = c < chunks;
-            uint4 a = make_uint4(0, 0, 0, 0), b = a;
-            if (active) {
-                a = ld_nc_v4(x + t * h + (int64_t)c * 16);
-                b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
-            }
-            float m = absmax16(a, b);
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            if (!active) continue;
-            const float amax_c = fmaxf(m, 1e-4f);
-            const float scale = __fdiv_rn(amax_c, 448.0f);
-            const float inv = __fdiv_rn(448.0f, amax_c);
-            const uint4 q = quant16(a, b, inv);
-            for (int j = 0; j < k; ++j) {
-                const int32_t row = s_dst[t * k + j];
-                if (row < 0) continue;
-                st_cs_v4(recv_x + (int64_t)row * h + (int64_t)c * 16, q);
-                if ((c & 7) == 0) recv_scale[(int64_t)row * nblk + (c >> 3)] = scale;
-            }
+    const int total = nt * chunks;   // a multiple of 8: a scale block never straddles tokens
+    for (int g0 = warp * 32; g0 < total; g0 += kThreads) {   // warp-uniform
+        const int g = g0 + lane;
+        const bool active = g < total;
+        const int tl = active ? g / chunks : 0, c = active ? g - tl * chunks : 0;
+        uint4 a = make_uint4(0, 0, 0, 0), b = a;
+        if (active) {
+            const uint16_t *src = x + (t0 + tl) * h + (int64_t)c * 16;
+            a = ld_nc_v4(src);
+            b = ld_nc_v4(src + 8);
+        }
+        float m = absmax16(a, b);
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        if (!active) continue;
+        const float amax_c = fmaxf(m, 1e-4f);
+        const float scale = __fdiv_rn(amax_c, 448.0f);
+        const float inv = __fdiv_rn(448.0f, amax_c);
+        const uint4 q = quant16(a, b, inv);
+        for (int j = 0; j < k; ++j) {
+            const int32_t row = s_dst[tl * k + j];
+            if (row < 0) continue;
+            st_cs_v4(recv_x + (int64_t)row * h + (int64_t)c * 16, q);
+            if ((c & 7) == 0) recv_scale[(int64_t)row * nblk + (c >> 3)] = scale;
         }
     }
 }
 
 // ------------------------------------------- fused layout + FP8 dispatch
 //
-// Prefill-sized batches: the layout and the FP8 dispatch in one cooperative
-// launch, one CTA of 768 threads per SM.  CTA b owns tokens [b T, b T + T)
-// both as a layout block and for the dispatch.  Warps 0-7 run the layout
-// block (its barriers are hardware barrier 1, 256 threads) and keep the
-// block's receive rows in shared memory; meanwhile warps 8-23 read the CTA's
-// first B tokens and stage their FP8 codes and scales in shared memory (the
-// dispatch's HBM reads overlap the layout's latency-bound exchange; 16 warps,
-// because the per-chunk quantisation is a dependent chain that needs several
-// warps per scheduler to hide).  After a full-block barrier the lanes of
-// warp 0 take (token, slot) pairs and hand the staged rows to the TMA engine,
-// one bulk copy per receive row (and one per scale row), so the rest of the
-// dispatch is HBM writes only.  It runs only when a CTA's whole share fits
-// in shared memory (B >= T: at hidden 7168 up to 28 tokens per CTA, 4144 on
-// 148 SMs); a second staging round could not overlap anything and measured
-// slower than the separate kernels.
+// Prefill-sized batches: the layout and the FP8 dispatch in one launch, one
+// CTA of 768 threads per SM.  CTA b owns tokens [b T, b T + T) both as a
+// replicated-count layout block and for the dispatch.
+//   1. All 24 warps read every id of the batch into the block's shared
+//      histograms (before / rest, designated ranks): the one phase whose cost
+//      grows with the batch, done first with every warp so it is short and
+//      nothing competes with it.
+//   2. Warps 0-7 then finish the layout block (own ranks, rows, outputs; their
+//      barriers are hardware barrier 1 with 256 threads) and keep the block's
+//      receive rows in shared memory, while warps 8-23 read the CTA's tokens
+//      and stage their FP8 codes and scales in shared memory, in token order.
+//      The tokens form up to kMaxGroups groups; every warp but warp 0 arrives
+//      on a group's hardware barrier (2 + g) once it has no chunk left in it.
+//   3. As soon as the rows are known, the lanes of warp 0 wait on each group's
+//      barrier in turn and hand its staged rows to the TMA engine, one bulk copy
+//      per receive row (and one per scale row), so the HBM writes of early
+//      tokens overlap the reads of later ones; warps 1-7 stage the CTA's last
+//      tokens.
+// At kernel start the TMA engine is also asked to bring the CTA's x rows into
+// L2 (one contiguous range), so that staging reads hit L2.
+// No CTA waits on another.  It runs only when a CTA's whole share fits in
+// shared memory (at hidden 7168 up to 28 tokens per CTA, 4144 on 148 SMs).
 
 constexpr int kLdThreads = 768;
-constexpr int kStageUnroll = 2;    // 16-value chunks per batch; two batches in registers
-constexpr int kLdColUnroll = 8;    // column-sum loads in flight (keeps the 768-thread kernel within 80 registers)
+constexpr int kStageUnroll = 2;    // thread-chunks per batch; two batches in registers
+constexpr int kGroupBar = 2;       // hardware barriers 2 .. 2 + kMaxGroups - 1: staged token groups
+constexpr int kMaxGroups = 14;
+// Share of a CTA's tokens staged by layout warps 1-7 once the layout is done
+// (they start a few microseconds after the 16 staging warps).
+constexpr int kLateShareNum = 5, kLateShareDen = 28;
+constexpr int64_t kPrefetchBytes = 32 * 1024;   // bytes per L2 prefetch instruction
+
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Tokens [group_begin(g), group_begin(g + 1)) of cnt form staging group g of ng.
+__device__ __forceinline__ int group_begin(int g, int cnt, int ng) { return (int)(((int64_t)g * cnt) / ng); }
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
-// Dynamic shared memory of the fused layout + dispatch kernel: the layout's
-// region, the block's receive rows (T k words), then B staged rows of h codes
+// Dynamic shared memory of the fused layout + dispatch kernel: the layout
+// block's region, its receive rows (T k words), then B staged rows of h codes
 // and h / 128 fp32 scales.
 __host__ __device__ __forceinline__ size_t ld_fixed_bytes(int k, int E, int R, int T) {
-    return align16(smem_words(0, k, E, R) * sizeof(int32_t) + (size_t)T * k * sizeof(int32_t));
+    return align16(rep_smem_words(T, E, R) * sizeof(int32_t) + (size_t)T * k * sizeof(int32_t));
 }
 __host__ __device__ __forceinline__ size_t ld_row_bytes(int h) { return (size_t)h + (size_t)(h >> 7) * 4; }
 
-// Quantise `cnt` tokens starting at global token t_first into the staged rows
-// (codes qbuf[t][h], scales sbuf[t][h / 128]).  Threads [th0, th0 + nth) take
-// part (th0, nth multiples of 32); the loop is uniform over them so every lane
-// joins the shuffles.  The arithmetic is the dispatch kernel's: block absmax,
-// amax_c = max(amax, 1e-4), scale = amax_c / 448 and inv = 448 / amax_c (IEEE
-// divisions), codes = e4m3_rn_satfinite(x * inv).
+// Quantise staged tokens: thread-chunks of kStageV consecutive values of one
+// token (one 16-byte load per 8 values), kStageLanes = 128 / kStageV lanes per
+// 128-value scale block, which combine their block maximum with xor-shuffles.
+// The arithmetic is the dispatch kernel's: block absmax, amax_c = max(amax,
+// 1e-4), scale = amax_c / 448 and inv = 448 / amax_c (IEEE divisions), codes =
+// e4m3_rn_satfinite(x * inv), written to qbuf[t][h]; the block's first lane
+// writes the scale to sbuf[t][h / 128].  (32 values per thread, with half the
+// shuffles and divisions per value, measured slower on B200: 72.6 against
+// 63 us for the whole kernel at 4096 tokens.)
+constexpr int kStageV = 16;
+constexpr int kStageLanes = 128 / kStageV;
+constexpr int kStageLoads = kStageV / 8;     // 16-byte loads per thread-chunk
+
 struct StageBatch {
-    uint4 a[kStageUnroll], b[kStageUnroll];
+    uint4 d[kStageUnroll][kStageLoads];
     int t[kStageUnroll], c[kStageUnroll];
 };
 
 // Issue the loads of the next kStageUnroll chunks of this thread ((t, c)
-// advanced by nth chunks per step).
+// advanced by nth chunks per step).  The loads allocate in L1: the two 16-byte
+// halves of a lane's 32-byte sector come from consecutive instructions.
 __device__ __forceinline__ void stage_load(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
                                            int chunks, int dt, int dc, int &t, int &c, StageBatch &B) {
 #pragma unroll
     for (int u = 0; u < kStageUnroll; ++u) {
         B.t[u] = t;
         B.c[u] = c;
-        B.a[u] = make_uint4(0, 0, 0, 0);
-        B.b[u] = B.a[u];
-        if (t < cnt) {
-            const uint16_t *src = x + (t_first + t) * h + (int64_t)c * 16;
-            B.a[u] = ld_nc_v4(src);
-            B.b[u] = ld_nc_v4(src + 8);
-        }
+        const uint16_t *src = x + (t_first + t) * h + (int64_t)c * kStageV;
+#pragma unroll
+        for (int i = 0; i < kStageLoads; ++i) B.d[u][i] = t < cnt ? ld_nc_l1_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
         t += dt;
         c += dc;
         if (c >= chunks) { c -= chunks; ++t; }
@@ -1194,59 +1310,85 @@ __device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch 
     const int nblk = h >> 7;
 #pragma unroll
     for (int u = 0; u < kStageUnroll; ++u) {
-        float m = absmax16(B.a[u], B.b[u]);
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kStageLoads; i += 2) m = fmaxf(m, absmax16(B.d[u][i], B.d[u][i + 1]));
+#pragma unroll
+        for (int o = kStageLanes / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         if (B.t[u] < cnt) {
             const float amax_c = fmaxf(m, 1e-4f);
             const float scale = __fdiv_rn(amax_c, 448.0f);
             const float inv = __fdiv_rn(448.0f, amax_c);
-            *reinterpret_cast<uint4 *>(qbuf + (size_t)B.t[u] * h + (size_t)B.c[u] * 16) =
-                quant16(B.a[u], B.b[u], inv);
-            if ((B.c[u] & 7) == 0) sbuf[B.t[u] * nblk + (B.c[u] >> 3)] = scale;
+            uint4 *dst = reinterpret_cast<uint4 *>(qbuf + (size_t)B.t[u] * h + (size_t)B.c[u] * kStageV);
+#pragma unroll
+            for (int i = 0; i < kStageLoads; i += 2) dst[i / 2] = quant16(B.d[u][i], B.d[u][i + 1], inv);
+            if ((B.c[u] & (kStageLanes - 1)) == 0) sbuf[B.t[u] * nblk + B.c[u] / kStageLanes] = scale;
         }
     }
 }
 
-__device__ void stage_fp8_rows(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
-                               uint8_t *qbuf, float *sbuf, int th0, int nth) {
-    const int chunks = h >> 4;
-    const int total = cnt * chunks;    // a multiple of 8: a scale group never straddles tokens
+// Stage tokens [tok_begin, tok_end) of the CTA's cnt tokens (global tokens
+// t_first + ...; see stage_quantise) with threads [th0, th0 + nth), and signal
+// the store issuer group by group: the CTA's tokens form ng groups, and a warp
+// arrives on barrier kGroupBar + g (bar_count threads in all) once its next
+// chunk lies past group g (a thread's chunks come in increasing order, and
+// lane 0's is the warp's lowest), after a proxy fence so that the bulk copies
+// see its codes.  Groups before the range are arrived on at once, those after
+// it at the end: every calling warp arrives on every group exactly once.
+__device__ void stage_fp8_rows_grouped(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
+                                       int tok_begin, int tok_end, uint8_t *qbuf, float *sbuf, int th0, int nth,
+                                       int ng, int bar_count) {
+    const int chunks = h / kStageV;    // a multiple of kStageLanes: a scale block never straddles tokens
+    const int q0 = tok_begin * chunks, q1 = tok_end * chunks;
     const int me = (int)threadIdx.x - th0;
+    const int wme = me & ~31;          // lane 0's offset
     // (token, chunk) of this thread's next chunk, advanced by nth per step
     const int dt = nth / chunks, dc = nth - dt * chunks;
-    int t = me / chunks, c = me - t * chunks;
+    int t = (q0 + me) / chunks, c = (q0 + me) - t * chunks;
+    int g_next = 0;                    // next group this warp arrives on
+    auto arrive_below = [&](int64_t next_min) {
+        while (g_next < ng && (int64_t)group_begin(g_next + 1, cnt, ng) * chunks <= next_min) {
+            fence_proxy_async();
+            bar_arrive(kGroupBar + g_next, bar_count);
+            ++g_next;
+        }
+    };
+    arrive_below((int64_t)q0 + wme);
     // two batches in registers: the next batch's loads are in flight while
     // the current one is quantised (uniform loop: every lane joins the shuffles)
     const int step = nth * kStageUnroll;
     StageBatch b0, b1;
-    stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b0);
-    for (int base = 0; base < total; base += 2 * step) {
-        const bool has1 = base + step < total, has2 = base + 2 * step < total;
-        if (has1) stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b1);
-        stage_quantise(h, cnt, b0, qbuf, sbuf);
+    if (q0 < q1) stage_load(x, h, t_first, tok_end, chunks, dt, dc, t, c, b0);
+    for (int base = q0; base < q1;) {
+        const bool has1 = base + step < q1;
+        if (has1) stage_load(x, h, t_first, tok_end, chunks, dt, dc, t, c, b1);
+        stage_quantise(h, tok_end, b0, qbuf, sbuf);
+        base += step;
+        arrive_below((int64_t)wme + base);
         if (!has1) break;
-        if (has2) stage_load(x, h, t_first, cnt, chunks, dt, dc, t, c, b0);
-        stage_quantise(h, cnt, b1, qbuf, sbuf);
+        const bool has2 = base + step < q1;
+        if (has2) stage_load(x, h, t_first, tok_end, chunks, dt, dc, t, c, b0);
+        stage_quantise(h, tok_end, b1, qbuf, sbuf);
+        base += step;
+        arrive_below((int64_t)wme + base);
+        if (!has2) break;
     }
+    arrive_below(INT64_MAX);
 }
 
-// Write staged tokens [tl, tl + cnt) of this CTA (staged rows 0..cnt) to their
-// receive rows: one bulk copy per (token, slot) with a row, issued by the
-// lanes of warp 0 (measured ~1% faster than spreading the issue over every
-// thread); scales by bulk copy when their row is a multiple of 16 bytes and
-// 16-byte aligned, else by plain stores.  Each issuing lane commits its own
-// bulk group.
-__device__ void store_fp8_rows(int k, int h, int tl, int cnt, const int32_t *s_dst, const uint8_t *qbuf,
+// Write staged tokens [t_begin, t_end) of this CTA to their receive rows: one
+// bulk copy per (token, slot) with a row, issued by the 32 lanes of the
+// calling warp; scales by bulk copy when their row is a multiple of 16 bytes
+// and 16-byte aligned, else by plain stores.  Each lane commits its own bulk
+// group.
+__device__ void issue_fp8_rows(int k, int h, int t_begin, int t_end, const int32_t *s_dst, const uint8_t *qbuf,
                                const float *sbuf, uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale,
                                bool scale_bulk) {
     const int nblk = h >> 7;
-    const int np = cnt * k;
-    if (threadIdx.x >= 32) return;
-    for (int p = threadIdx.x; p < np; p += 32) {
+    const int lane = threadIdx.x & 31;
+    for (int p = t_begin * k + lane; p < t_end * k; p += 32) {
         const int t = p / k;
-        const int32_t row = s_dst[tl * k + p];
+        const int32_t row = s_dst[p];
         if (row < 0) continue;
         bulk_store(recv_x + (int64_t)row * h, qbuf + (size_t)t * h, (uint32_t)h);
         if (scale_bulk) {
@@ -1261,38 +1403,56 @@ __device__ void store_fp8_rows(int k, int h, int tl, int cnt, const int32_t *s_d
 template <int CH>
 __global__ void __launch_bounds__(kLdThreads, 1)
 layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int T,
-                           int B, uint64_t *flags, uint32_t salt, int32_t *ws_e, int32_t *ws_r,
-                           int32_t *__restrict__ tokens_per_expert, int32_t *__restrict__ tokens_per_rank,
-                           uint8_t *__restrict__ in_rank, int32_t *__restrict__ expert_offset,
-                           int32_t *__restrict__ max_count, int32_t *__restrict__ dst_pos,
-                           int32_t *__restrict__ recv_src, int64_t recv_rows, const uint16_t *__restrict__ x,
-                           int h, uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, int scale_bulk,
-                           uint32_t *status) {
+                           int B, int vec, int32_t *__restrict__ tokens_per_expert,
+                           int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
+                           int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
+                           int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
+                           const uint16_t *__restrict__ x, int h, uint8_t *__restrict__ recv_x,
+                           float *__restrict__ recv_scale, int scale_bulk, uint32_t *status) {
     extern __shared__ __align__(128) int32_t smem_ld[];
     __shared__ int32_t scan_tmp[32];
-    __shared__ int s_ok;
-    const Smem s = carve(0, smem_ld, k, E, R);
-    int32_t *s_dst = smem_ld + smem_words(0, k, E, R);
+    const Smem s = carve_rep(smem_ld, T, E, R);
+    int32_t *s_dst = smem_ld + rep_smem_words(T, E, R);
     uint8_t *qbuf = reinterpret_cast<uint8_t *>(smem_ld) + ld_fixed_bytes(k, E, R, T);
     float *sbuf = reinterpret_cast<float *>(qbuf + (size_t)B * h);
     const int64_t t0 = (int64_t)blockIdx.x * T;
     const int nt = t0 < n ? (int)(n - t0 < T ? n - t0 : T) : 0;
     const int cnt0 = nt < B ? nt : B;   // == nt: the host launches this kernel only when B >= T
-    if (threadIdx.x < kThreads) {
-        const bool ok = layout_block<false, CH, kLdColUnroll, true>(idx, n, k, E, R, cap, E, E / R, T, flags, salt,
-                                                ws_e, ws_r,
-                                                tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                                                max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp,
-                                                s_dst);
-        if (threadIdx.x == 0) s_ok = ok;
-    } else {
-        stage_fp8_rows(x, h, t0, cnt0, qbuf, sbuf, kThreads, kLdThreads - kThreads);
-        fence_proxy_async();
+    const int ng = cnt0 < kMaxGroups ? (cnt0 > 0 ? cnt0 : 1) : kMaxGroups;
+    const int split = cnt0 - (cnt0 * kLateShareNum) / kLateShareDen;   // warps 1-7 stage [split, cnt0)
+    griddep_wait();   // ids and x may come from the kernels just before, which may still read our outputs
+    if (threadIdx.x < 32 && cnt0 > 0) {
+        // the CTA's x rows are one contiguous range: the TMA engine streams it from
+        // HBM into L2 while the ids are scanned, so the staging loads hit L2
+        const char *src = reinterpret_cast<const char *>(x + t0 * h);
+        const int64_t bytes = (int64_t)cnt0 * h * 2;
+        for (int64_t off = (int64_t)threadIdx.x * kPrefetchBytes; off < bytes; off += 32 * kPrefetchBytes)
+            prefetch_l2_bulk(src + off, (uint32_t)(bytes - off < kPrefetchBytes ? bytes - off : kPrefetchBytes));
     }
+    PairsT<CH> P;
+    bool bad = false;
+    if (threadIdx.x < kThreads) bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight
+    rep_zero<kLdThreads>(T, E, R, s);
     __syncthreads();
-    if (!s_ok) return;   // the inter-block wait timed out (reported); nothing is written
-    store_fp8_rows(k, h, 0, cnt0, s_dst, qbuf, sbuf, recv_x, recv_scale, scale_bulk != 0);
-    bulk_wait_all();
+    rep_scan<kLdThreads>(idx, n, k, E, R, t0, vec != 0, s);
+    __syncthreads();
+    if (threadIdx.x < kThreads) {
+        rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                       max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
+        lsync();   // every row of the block is in s_dst
+        if (threadIdx.x < 32) {
+            for (int g = 0; g < ng; ++g) {
+                bar_sync(kGroupBar + g, kLdThreads);   // group g is staged
+                issue_fp8_rows(k, h, group_begin(g, cnt0, ng), group_begin(g + 1, cnt0, ng), s_dst, qbuf, sbuf,
+                               recv_x, recv_scale, scale_bulk != 0);
+            }
+            bulk_wait_all();
+        } else {   // warps 1-7, free after the layout: the CTA's last tokens
+            stage_fp8_rows_grouped(x, h, t0, cnt0, split, cnt0, qbuf, sbuf, 32, kThreads - 32, ng, kLdThreads);
+        }
+    } else {
+        stage_fp8_rows_grouped(x, h, t0, cnt0, 0, split, qbuf, sbuf, kThreads, kLdThreads - kThreads, ng, kLdThreads);
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1366,6 +1526,19 @@ int cluster_ctas_for(int64_t n, int k, int nkeys, int R) {
     return ok == 1 ? (int)C : 0;
 }
 
+// Blocks of the replicated-count layout for n tokens (one chunk per warp, T =
+// tokens_per_block(k, 1) tokens per block), or 0 when it does not apply: more
+// than kRepMaxPairs pairs, more than 32 designated ranks per block, or more
+// shared memory than a kernel gets without opting in.
+int rep_grid(int64_t n, int k, int E, int R) {
+    if (n * k > kRepMaxPairs) return 0;
+    const int T = tokens_per_block(k, 1);
+    const int64_t G = n > 0 ? (n + T - 1) / T : 1;
+    if (G > 1 && rep_designated(0, (int)G, R) > 32) return 0;
+    if (rep_smem_words(T, E, R) * sizeof(int32_t) > kSmemDefault) return 0;
+    return (int)G;
+}
+
 template <bool kRankKeys>
 bool fused_fits(int64_t n, int k, int nkeys, int R) {
     const WsLayout w = ws_layout(n, k, nkeys, R);
@@ -1409,7 +1582,7 @@ LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
     if (num_sms > 0 && num_sms < sms) sms = num_sms;
     if (n <= 0 || sms <= 0 || h <= 0 || h % 128 != 0) return r;
     if (n * k < 64 * (int64_t)sms) return r;   // small batches: a few CTAs would carry the whole dispatch
-    if (E % 8 != 0) return r;                   // its count rows are 16-bit, 8 per 16-byte load
+    if (n * k > kRepMaxPairs) return r;         // every CTA reads all ids
     int64_t T = (n + sms - 1) / sms;
     const int t_min = 64 / k > 0 ? 64 / k : 1;
     if (T < t_min) T = t_min;
@@ -1419,6 +1592,7 @@ LdShape ld_shape(int64_t n, int k, int E, int R, int h, int num_sms) {
     r.CH = pairs <= 256 ? 1 : (pairs <= 512 ? 2 : 4);
     r.G = (int)((n + T - 1) / T);
     if (r.G > kLdMaxBlocks) return r;
+    if (rep_designated(0, r.G, R) > 32) return r;
     const int optin = optin_smem_bytes();
     if (optin <= 0) return r;
     const size_t avail = optin > 1024 ? (size_t)optin - 1024 : 0;   // room for the static shared memory
@@ -1462,7 +1636,7 @@ bool ld_launchable(const LdShape &sh) {
         std::lock_guard<std::mutex> lk(g_mu);
         if (g_ld_occ_n < 64) g_ld_occ[g_ld_occ_n++] = {dev, CH, sh.smem, occ};
     }
-    return (int64_t)occ * device_sm_count() >= sh.G;
+    return occ >= 1;   // no co-residency needed: the CTAs never wait on one another
 }
 
 bool ld_fits(const LdShape &sh) {
@@ -1478,32 +1652,15 @@ template <int CH>
 cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                      const uint16_t *x, int h, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
                      uint8_t *in_rank, int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
-                     int32_t *recv_src, uint8_t *recv_x, float *recv_scale, void *ws, uint32_t *status,
-                     cudaStream_t stream) {
-    const WsLayout w = ws_layout_blocks(sh.G, E, R);
-    uint64_t *flags = static_cast<uint64_t *>(ws);
-    int32_t *ws_e = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.e_off);
-    int32_t *ws_r = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + w.r_off);
+                     int32_t *recv_src, uint8_t *recv_x, float *recv_scale, uint32_t *status, cudaStream_t stream) {
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
     const int scale_bulk = ((h >> 7) % 4 == 0) && (reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)sh.G);
-    cfg.blockDim = dim3(kLdThreads);
-    cfg.dynamicSmemBytes = sh.smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t err = cudaLaunchKernelEx(
-        &cfg, layout_dispatch_fp8_kernel<CH>, idx, n, k, E, R, cap, sh.T, sh.B, flags, next_salt(), ws_e, ws_r,
-        tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src, recv_rows, x, h,
-        recv_x, recv_scale, scale_bulk, status);
-    if (err == cudaSuccess) return CGL_OK;
-    if (err != cudaErrorCooperativeLaunchTooLarge) return CGL_ECUDA;
-    cudaGetLastError();   // fewer SMs free than the occupancy query counted: the caller splits the work
-    return CGL_ENOTIMPL;
+    const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+    const cudaError_t err = launch_pdl(layout_dispatch_fp8_kernel<CH>, dim3((unsigned)sh.G), dim3(kLdThreads), sh.smem,
+                                       stream, idx, n, k, E, R, cap, sh.T, sh.B, vec, tokens_per_expert,
+                                       tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src,
+                                       recv_rows, x, h, recv_x, recv_scale, scale_bulk, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
 }  // namespace
@@ -1511,9 +1668,7 @@ cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, in
 size_t layout_workspace_bytes(int64_t n, int k, int E, int R) { return ws_layout(n, k, E, R).bytes; }
 
 size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
-    const int64_t blocks = n < 1 ? 1 : (n < kLdMaxBlocks ? n : kLdMaxBlocks);
-    const size_t fused = ws_layout_blocks(blocks, E, R).bytes, split = ws_layout(n, k, E, R).bytes;
-    return fused > split ? fused : split;
+    return ws_layout(n, k, E, R).bytes;   // the fused kernel needs none; the split path the layout's
 }
 
 bool layout_dispatch_fused_fits(int64_t n, int k, int E, int R, int h, int num_sms) {
@@ -1528,24 +1683,17 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       cudaStream_t stream) {
     const LdShape sh = ld_shape(n, k, E, R, h, num_sms);
     if (ld_fits(sh)) {
-        cgl_status st = CGL_ECUDA;
         switch (sh.CH) {
             case 1:
-                st = ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                  stream);
-                break;
+                return ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
             case 2:
-                st = ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                  stream);
-                break;
+                return ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
             default:
-                st = ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                  expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, ws, status,
-                                  stream);
+                return ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
         }
-        if (st != CGL_ENOTIMPL) return st;   // CGL_ENOTIMPL: the cooperative launch was refused
     }
     const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
                                         expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
@@ -1558,7 +1706,7 @@ bool layout_needs_smem_optin(int E, int R, int k) {
     return smem_words(0, k, E, R) * sizeof(int32_t) > kSmemDefault;
 }
 
-bool layout_fused_fits(int64_t n, int k, int E, int R) { return fused_fits<false>(n, k, E, R); }
+bool layout_fused_fits(int64_t n, int k, int E, int R) { return rep_grid(n, k, E, R) > 0 || fused_fits<false>(n, k, E, R); }
 
 template <bool kRankKeys, int CH>
 cgl_status launch_layout_ch(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
@@ -1617,6 +1765,24 @@ cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, i
                               int32_t *key_offset, int32_t *max_count, int32_t *dst_pos,
                               int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
     const int nkeys = kRankKeys ? R : E_ids;
+    if constexpr (!kRankKeys) {
+        const int G = rep_grid(n, k, E_ids, R);
+        if (G > 0) {
+            const int T = tokens_per_block(k, 1);
+            const int64_t recv_rows = cap > 0 ? (int64_t)E_ids * cap : n * k;
+            const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+            const size_t smem = rep_smem_words(T, E_ids, R) * sizeof(int32_t);
+            const cudaError_t err =
+                n * k > kRepWidePairs
+                    ? launch_pdl(layout_rep_kernel<1, kRepThreads>, dim3((unsigned)G), dim3(kRepThreads), smem, stream,
+                                 idx, n, k, E_ids, R, cap, vec, tokens_per_key, tokens_per_rank, in_rank, key_offset,
+                                 max_count, dst_pos, recv_src, recv_rows, status)
+                    : launch_pdl(layout_rep_kernel<1, kThreads>, dim3((unsigned)G), dim3(kThreads), smem, stream, idx,
+                                 n, k, E_ids, R, cap, vec, tokens_per_key, tokens_per_rank, in_rank, key_offset,
+                                 max_count, dst_pos, recv_src, recv_rows, status);
+            return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+        }
+    }
     const int C = cluster_ctas_for<kRankKeys>(n, k, nkeys, R);
     if (C > 0) {
         cudaLaunchConfig_t cfg = {};
@@ -1674,8 +1840,30 @@ cgl_status launch_wait_probe(uint64_t *ws, int nflags, uint32_t *status, cudaStr
     return cudaGetLastError() == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
+// Launch shape of the fused decode kernel: G CTAs of T tokens (at most one CTA
+// per SM in use, and T k <= 1024 pairs); one CTA for everything when more
+// CTAs would give one of them more than 32 designated ranks.
+struct DecodeShape {
+    int G, T, CH;
+};
+DecodeShape decode_shape(int64_t n, int k, int R, int use_sms) {
+    DecodeShape d;
+    const int64_t g = n < 1 ? 1 : (n < use_sms ? n : use_sms);
+    d.T = n < 1 ? 1 : (int)((n + g - 1) / g);
+    d.G = n < 1 ? 1 : (int)((n + d.T - 1) / d.T);
+    if (d.G > 1 && rep_designated(0, d.G, R) > 32) {
+        d.G = 1;
+        d.T = n < 1 ? 1 : (int)n;
+    }
+    const int64_t pairs = (int64_t)d.T * k;
+    d.CH = pairs <= 256 ? 1 : (pairs <= 512 ? 2 : 4);
+    return d;
+}
+
 size_t decode_fused_smem_bytes(int64_t n, int k, int E, int R) {
-    return (smem_words(0, k, E, R) + (size_t)(n * k)) * sizeof(int32_t);
+    // the largest T any launch shape uses is n (a single CTA)
+    const int T = n < 1 ? 1 : (int)n;
+    return (rep_smem_words(T, E, R) + (size_t)T * k) * sizeof(int32_t);
 }
 
 cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int E, int R, int cap,
@@ -1688,11 +1876,26 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
     const int sms = device_sm_count();
     if (sms <= 0) return CGL_ECUDA;
     const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
-    const int64_t grid = n < 1 ? 1 : (n < use_sms ? n : use_sms);
-    const cudaError_t err = launch_pdl(decode_fused_kernel, dim3((unsigned)grid), dim3(kThreads),
-                                       decode_fused_smem_bytes(n, k, E, R), stream, idx, n, k, E, R, cap, x, h,
-                                       tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
-                                       dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+    const DecodeShape d = decode_shape(n, k, R, use_sms);
+    const size_t smem = (rep_smem_words(d.T, E, R) + (size_t)d.T * k) * sizeof(int32_t);
+    const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+    cudaError_t err;
+    switch (d.CH) {
+        case 1:
+            err = launch_pdl(decode_fused_kernel<1>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
+                             R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+            break;
+        case 2:
+            err = launch_pdl(decode_fused_kernel<2>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
+                             R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+            break;
+        default:
+            err = launch_pdl(decode_fused_kernel<4>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
+                             R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+    }
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 

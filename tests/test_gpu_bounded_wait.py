@@ -72,11 +72,12 @@ def test_graph_replay_after_a_timed_out_exchange_gets_a_new_tag(oracle_mod):
     flag published with the tag of the generation word's next launch), run
     the wait's timeout path on it, then replay with new ids: the replay must
     not take those flags for its own."""
-    a, b = W.make_inputs("prefill", 2), W.make_inputs("prefill", 3)
+    a, b = W.make_inputs("skewed", 2), W.make_inputs("skewed", 3)
     E, R = 256, 64
     n, k = a.topk_idx.shape
+    assert n * k > 32768                                      # past the replicated-count layout:
     assert cgl.layout_kernel_count(n, k, E, R) == 1          # the cooperative exchange
-    ws = torch.empty(cgl.layout_workspace_bytes(n, k, E, R), dtype=torch.uint8, device=dev())
+    ws = torch.zeros(cgl.layout_workspace_bytes(n, k, E, R), dtype=torch.uint8, device=dev())
     idx = i32(a.topk_idx)
     st = cgl.new_status(dev())
     lay = cgl.get_layout(idx, E, R, workspace=ws, status=st)
@@ -89,7 +90,7 @@ def test_graph_replay_after_a_timed_out_exchange_gets_a_new_tag(oracle_mod):
     _assert_layout(oracle_mod, lay, a.topk_idx, E, R)
     words = _words(ws)
     gen = int(words[0].item())
-    nb = (n + 63) // 64                                       # 64 tokens per block at this size
+    nb = (n + 127) // 128                                     # 128 tokens per block at this size
     flags = words[1:1 + nb]
     assert torch.all(flags == flags[0]).item() and (int(flags[0].item()) & 0xFFFFFFFF) == (gen & 0xFFFFFFFF)
     # the state a replay that timed out before advancing would leave: generation
@@ -113,11 +114,15 @@ def test_graph_replay_after_a_timed_out_exchange_gets_a_new_tag(oracle_mod):
 def test_layout_calls_are_right_on_any_workspace_contents(oracle_mod, fill):
     """A workspace with a generation word g, flags equal to the tag scheme an
     earlier build used for generation g + 1, and garbage count rows; or all
-    zero, or all ones: both exchange calls match the oracle bit for bit."""
-    a = W.make_inputs("prefill", 5)
+    zero, or all ones: both calls that exchange counts through it (the layout,
+    and the layout + FP8 dispatch, which at 16384 tokens runs the layout and
+    dispatch kernels) match the oracle bit for bit."""
+    a = W.make_inputs("skewed", 5)
     E, R = 256, 64
     n, k = a.topk_idx.shape
     wl = a.workload
+    assert cgl.layout_kernel_count(n, k, E, R) == 1
+    assert cgl.layout_dispatch_kernel_count(n, k, E, R, wl.hidden) == 2
     nbytes = max(cgl.layout_workspace_bytes(n, k, E, R), cgl.layout_dispatch_workspace_bytes(n, k, E, R))
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev())
     words = _words(ws)

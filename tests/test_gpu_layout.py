@@ -178,3 +178,34 @@ def test_layout_graph_replays_with_changing_ids(oracle_mod, name):
         assert np.array_equal(lay.recv_src.cpu().numpy(), ref.recv_src)
         assert np.array_equal(lay.tokens_per_rank.cpu().numpy(), ref.tokens_per_rank)
     del g
+
+
+def test_layout_replicated_counts_with_unaligned_ids(oracle_mod):
+    """Ids that start 4 bytes past a 16-byte boundary: the replicated-count
+    layout reads them one by one instead of as int4."""
+    rng = np.random.default_rng(21)
+    n, k, E, R = 3000, 8, 256, 64
+    a = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    a[rng.random((n, k)) < 0.04] = -1
+    buf = torch.empty(n * k + 1, dtype=torch.int32, device=dev())
+    idx = buf[1:].view(n, k)
+    assert idx.data_ptr() % 16 == 4
+    idx.copy_(torch.from_numpy(a))
+    st = cgl.new_status(dev())
+    lay = cgl.get_layout(idx, E, R, status=st)
+    torch.cuda.synchronize()
+    ref = oracle_mod.get_layout(a, E, R)
+    for f in ("tokens_per_expert", "tokens_per_rank", "is_token_in_rank", "expert_offset", "dst_pos", "recv_src"):
+        assert np.array_equal(getattr(lay, f).cpu().numpy(), getattr(ref, f)), f
+    assert st.item() == 0
+
+
+@pytest.mark.parametrize("n,k,E,R", [(64, 8, 256, 128), (250, 4, 512, 256)])
+def test_layout_cluster_path_many_ranks(oracle_mod, n, k, E, R):
+    """More ranks than 32 per block of the replicated-count layout: these small
+    batches take the thread-block-cluster layout instead."""
+    rng = np.random.default_rng(n + R)
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    idx[rng.random((n, k)) < 0.05] = -1
+    lay, _ = run_both(oracle_mod, idx, E, R, 0)
+    run_both(oracle_mod, idx, E, R, max(1, int(lay.max_count.item()) - 1))

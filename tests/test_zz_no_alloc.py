@@ -78,27 +78,31 @@ def _oracle_check(oracle_mod, got, idx_np, E, R, cap):
 def test_noalloc_matches_oracle_and_get_layout_on_calls_in_a_row(oracle_mod):
     """Consecutive calls of different shapes share the scratch array: each later
     call runs on what the one before left in it (generation word, flags and count
-    rows of another block count, E and R).  Every call takes the path that
-    exchanges counts through the array (several layout blocks), except the
-    padded decode call, which needs none.  Each output is compared bit for bit
-    with the oracle and with cgl_get_layout."""
+    rows of another block count, E and R).  Calls above 32768 (token, slot) pairs
+    exchange counts through the array (cooperative blocks); the prefill-sized
+    and decode calls in between need no scratch and check that the array's
+    contents do not matter to them.  Each output is compared bit for bit with
+    the oracle and with cgl_get_layout."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    pre = W.make_inputs("prefill", 0)           # 64 blocks of 64 tokens, E=256, R=64
-    skw = W.make_inputs("skewed", 0)            # 128 blocks of 128 tokens, E=256, R=32 (ranks of 8 experts)
+    pre = W.make_inputs("prefill", 0)
+    skw = W.make_inputs("skewed", 0)
     dec = W.make_inputs("decode", 0)
-    cap_pre = oracle_mod.get_layout(pre.topk_idx, 256, 64).max_count
+    s9 = np.ascontiguousarray(skw.topk_idx[:9000])
+    cap_s9 = oracle_mod.get_layout(s9, 256, 64).max_count
     cap_dec = oracle_mod.get_layout(dec.topk_idx, 256, 32).max_count
     cases = [
-        (pre.topk_idx, 256, 64, 0),
-        (skw.topk_idx, 256, 32, 0),
-        (pre.topk_idx, 256, 64, cap_pre - 3),   # padded, some experts overflow (CGL_ECAPACITY)
+        (skw.topk_idx, 256, 64, 0),             # 128 blocks of 128 tokens
+        (skw.topk_idx, 256, 32, 0),             # same blocks, other R
+        (s9, 256, 64, cap_s9 - 3),              # 71 blocks, padded, some experts overflow (CGL_ECAPACITY)
+        (pre.topk_idx, 256, 64, 0),             # replicated counts: no scratch
         (dec.topk_idx, 256, 32, cap_dec),
-        (pre.topk_idx[:1500], 256, 64, 0),      # 47 blocks of 32 tokens
-        (pre.topk_idx, 256, 64, 0),
+        (skw.topk_idx[:5000], 256, 64, 0),      # 40 blocks
+        (skw.topk_idx, 256, 64, 0),
     ]
     for idx_np, E, R, c in cases:
-        idx = torch.from_numpy(np.ascontiguousarray(idx_np)).to(dev)
+        idx_np = np.ascontiguousarray(idx_np)
+        idx = torch.from_numpy(idx_np).to(dev)
         got, st = _noalloc(idx, E, R, c)
         ref, st_ref = _reference(idx, E, R, c)
         torch.cuda.synchronize()
