@@ -40,20 +40,21 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes per launch read by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
 # for the kernels at the 4096-token prefill shape, with the sha256 of the kernel
-# source they were taken on; a changed source reports traffic null.  (The
-# "layout" record was carried over edits of layout.cu that did not touch
-# layout_fused_kernel: host-side caches, launch fallbacks and the fused
-# dispatch's store loop and count-row format.)
+# source and the shared device header it was taken on; a changed source
+# reports traffic null.
 NCU_TRAFFIC = {
-    "combine": {"bytes": 507180800, "src_sha": "ecb3bf8c62c6e9dc"},
-    "dispatch_fp8": {"bytes": 242248448, "src_sha": "34b4b5d953b8ca4c"},
-    "layout": {"bytes": 206080, "src_sha": "8cdb38836f26e97a"},
+    "combine": {"bytes": 507093760, "src_sha": "e63c09f116de7be3"},
+    "dispatch_fp8": {"bytes": 243200256, "src_sha": "6c478e0bec1a7510"},
+    "layout+dispatch_fp8": {"bytes": 250198016, "src_sha": "909cacef0c241f29"},
+    "layout": {"bytes": 217600, "src_sha": "909cacef0c241f29"},
 }
 
 
 def _src_sha(name: str) -> str:
-    p = os.path.join(ROOT, "combine_get_layout_02_b200", "csrc", name)
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in (name, "common.cuh"):
+        h.update(open(os.path.join(ROOT, "combine_get_layout_02_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, src: str):
@@ -757,18 +758,22 @@ def run_ours(args):
     peak, peak_src = hbm_peak()
     alone = time_alone(step, min(args.steps, 200), peak)
     status_bits = sorted(set(status_bits) | set(step.cgl.status_bits(step.status)))
+    srcs = {"combine": "combine.cu", "dispatch_fp8": "dispatch.cu", "dispatch_bf16": "dispatch.cu",
+            "layout": "layout.cu", "layout+dispatch_fp8": "layout.cu", "combine_backward": "combine_backward.cu"}
+    # the traffic records were taken at the prefill shape, expert-keyed path
+    at_prefill = (wl.name == "prefill" and wl.num_tokens == W.WORKLOADS["prefill"].num_tokens and not args.dedup)
     kernels = {}
     for (name, launches, nbytes), t in zip(phases, per_phase):
         gbs = nbytes / (t * 1e-3) / 1e9
         kernels[name] = {"us": t * 1e3, "launches_per_step": launches, "bytes": nbytes,
-                         "gbs": gbs, "frac_of_peak": gbs / peak}
+                         "gbs": gbs, "frac_of_peak": gbs / peak,
+                         "traffic": traffic_for(name, srcs.get(name, "layout.cu")) if at_prefill else None}
     dom = max(phases, key=lambda p: p[2])[0]
-    src = {"combine": "combine.cu", "dispatch_fp8": "dispatch.cu", "dispatch_bf16": "dispatch.cu",
-           "layout": "layout.cu", "layout+dispatch_fp8": "layout.cu",
-           "combine_backward": "combine_backward.cu"}.get(dom, "layout.cu")
+    src = srcs.get(dom, "layout.cu")
     roof = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["gbs"], "peak": peak,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy read+write)" if peak_src == "measured" else "fallback 6.65 TB/s",
-            "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "traffic": traffic_for(dom, src),
+            "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
+            "traffic": traffic_for(dom, src) if at_prefill else None,
             "bytes_per_launch": kernels[dom]["bytes"],
             "timing": ("in the step: CUDA events on the launching stream around each launch of the kernel over "
                        "the K steps of the instrumented pass (the gap the events add included)")}
