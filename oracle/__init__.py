@@ -54,7 +54,9 @@ def lib():
                                              P, P, P, P, P]
         L.oracle_get_rank_layout.restype = C.c_int
         L.oracle_dispatch_fp8.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P, P]
+        L.oracle_dispatch_fp8_pow2.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P, P]
         L.oracle_dispatch_fp8.restype = None
+        L.oracle_dispatch_fp8_pow2.restype = None
         L.oracle_dispatch_bf16.argtypes = [P, C.c_int64, C.c_int, C.c_int, P, P]
         L.oracle_dispatch_bf16.restype = None
         L.oracle_combine_backward.argtypes = [P, P, P, P, C.c_int64, C.c_int, C.c_int, P, P]
@@ -156,10 +158,12 @@ def get_rank_layout(topk_idx: np.ndarray, num_experts: int, num_ranks: int, capa
     return RankLayout(tpr, off, int(mx[0]), dst, src, int(flags))
 
 
-def dispatch_fp8(x: np.ndarray, dst_pos: np.ndarray, num_rows: int):
+def dispatch_fp8(x: np.ndarray, dst_pos: np.ndarray, num_rows: int, pow2_scales: bool = False):
     """Returns (recv_x uint8 [num_rows, H], recv_scale fp32 [num_rows, H/128]).
 
-    Rows that receive no copy are zero (the CUDA path leaves them unwritten)."""
+    pow2_scales: power-of-two (UE8M0) scales, scale = the smallest 2^e with
+    448 * 2^e >= amax_c, inv = 2^-e.  Rows that receive no copy are zero (the
+    CUDA path leaves them unwritten)."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     dst = np.ascontiguousarray(dst_pos, dtype=np.int32)
     n, h = x.shape
@@ -168,7 +172,8 @@ def dispatch_fp8(x: np.ndarray, dst_pos: np.ndarray, num_rows: int):
         raise ValueError("hidden must be a multiple of 128 for FP8 dispatch")
     rx = np.zeros((num_rows, h), np.uint8)
     rs = np.zeros((num_rows, h // 128), np.float32)
-    lib().oracle_dispatch_fp8(_p(x), n, h, k, _p(dst), _p(rx), _p(rs))
+    fn = lib().oracle_dispatch_fp8_pow2 if pow2_scales else lib().oracle_dispatch_fp8
+    fn(_p(x), n, h, k, _p(dst), _p(rx), _p(rs))
     return rx, rs
 
 

@@ -312,6 +312,56 @@ void oracle_dispatch_fp8(const uint16_t *x, int64_t N, int H, int k, const int32
     }
 }
 
+/*
+ * FP8 dispatch with power-of-two (UE8M0) scales.  Reading: the variant of the
+ * dispatch above whose per-block scale is restricted to a power of two, as an
+ * 8-bit exponent-only (UE8M0) scale format can hold: scale = 2^e for the
+ * smallest integer e with 448 * 2^e >= amax_c (the block's largest value then
+ * maps to at most 448, so nothing saturates), inv = 2^-e, q = e4m3(x * inv).
+ * The scale is stored as the binary32 value 2^e (its biased exponent field is
+ * the UE8M0 code).  e is found by the plain search below: 448 * 2^e is exact
+ * in binary32 over the range searched, so each comparison is exact.
+ */
+static float pow2_scale_exponent_search(float amax_c, int *e_out) {
+    int e = -40;                          /* 448 * 2^-40 < 1e-4 <= amax_c */
+    while (ldexpf(448.0f, e) < amax_c) ++e;
+    *e_out = e;
+    return ldexpf(1.0f, e);
+}
+
+void oracle_dispatch_fp8_pow2(const uint16_t *x, int64_t N, int H, int k, const int32_t *dst_pos,
+                              uint8_t *recv_x, float *recv_scale) {
+    int nb = H / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        uint8_t q[H > 0 ? H : 1];
+        float sc[nb > 0 ? nb : 1];
+        for (int b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int i = 0; i < 128; ++i) {
+                float v = fabsf(bf16_to_f32(x[t * H + b * 128 + i]));
+                if (v > amax) amax = v;
+            }
+            float amax_c = amax > 1e-4f ? amax : 1e-4f;
+            int e;
+            float scale = pow2_scale_exponent_search(amax_c, &e);
+            float inv = ldexpf(1.0f, -e);
+            for (int i = 0; i < 128; ++i) {
+                float v = bf16_to_f32(x[t * H + b * 128 + i]);
+                float prod = v * inv;
+                q[b * 128 + i] = oracle_e4m3_encode(prod);
+            }
+            sc[b] = scale;
+        }
+        for (int j = 0; j < k; ++j) {
+            int32_t row = dst_pos[t * k + j];
+            if (row < 0) continue;
+            memcpy(recv_x + (int64_t)row * H, q, (size_t)H);
+            memcpy(recv_scale + (int64_t)row * nb, sc, sizeof(float) * (size_t)nb);
+        }
+    }
+}
+
 /* BF16 dispatch (and the combine-backward re-dispatch of gradient rows):
  * row t is copied bit for bit to each receive row dst_pos[t, j] >= 0. */
 void oracle_dispatch_bf16(const uint16_t *x, int64_t N, int H, int k, const int32_t *dst_pos,
