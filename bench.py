@@ -176,8 +176,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- steps
 
-def workload_label(wl: W.Workload, dedup: bool = False) -> str:
+def workload_label(wl: W.Workload, dedup: bool = False, pow2: bool = False) -> str:
     tail = "; per-rank deduplicated dispatch (one copy per token and rank)" if dedup else ""
+    tail += "; power-of-two (UE8M0) FP8 scales" if pow2 and wl.fp8 else ""
     return f"{wl.name}: {wl.description}{tail}"
 
 
@@ -185,13 +186,14 @@ class GpuStep:
     """Device buffers for one workload and the launch sequence of one step."""
 
     def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False, full_backward: bool = False,
-                 fused_decode: bool = False, split_layout: bool = False):
+                 fused_decode: bool = False, split_layout: bool = False, pow2_scales: bool = False):
         import torch
 
         import combine_get_layout_02_b200 as cgl
 
         self.cgl, self.torch, self.wl, self.dev = cgl, torch, wl, device
         self.dedup = dedup
+        self.pow2 = pow2_scales
         self.full_backward = full_backward and wl.with_grad and not dedup
         self.fused_decode = fused_decode and wl.fp8 and not dedup
         # FP8 steps call cgl_layout_dispatch_fp8 (one cooperative kernel when it
@@ -300,14 +302,15 @@ class GpuStep:
         rec()
         if self.fused_decode:
             cgl.decode_dispatch_fp8(self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x,
-                                    recv_scale=self.recv_scale, status=self.status)
+                                    recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2)
             rec()
             cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
             rec()
             return
         if self.layout_dispatch:
             cgl.layout_dispatch_fp8(self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x,
-                                    recv_scale=self.recv_scale, workspace=self.ws, status=self.status)
+                                    recv_scale=self.recv_scale, workspace=self.ws, status=self.status,
+                                    pow2_scales=self.pow2)
             rec()
             cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
             rec()
@@ -317,7 +320,7 @@ class GpuStep:
             rec()
             if wl.fp8:
                 cgl.dispatch_fp8(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
-                                 recv_scale=self.recv_scale, status=self.status)
+                                 recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2)
             else:
                 cgl.dispatch_bf16(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
                                   status=self.status)
@@ -333,7 +336,7 @@ class GpuStep:
         rec()
         if wl.fp8:
             cgl.dispatch_fp8(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
-                             recv_scale=self.recv_scale, status=self.status)
+                             recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2)
         else:
             cgl.dispatch_bf16(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
                               status=self.status)
@@ -369,12 +372,12 @@ class GpuStep:
         calls = [("layout", lay_call, b["layout"])]
         if wl.fp8:
             calls.append(("dispatch_fp8", lambda: cgl.dispatch_fp8(self.x, dst, rows, recv_x=self.recv_x,
-                                                                   recv_scale=self.recv_scale, status=self.status),
+                                                                   recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2),
                           b["dispatch_fp8"]))
             if self.layout_dispatch:
                 calls.append(("layout+dispatch_fp8", lambda: cgl.layout_dispatch_fp8(
                     self.idx, self.x, E, R, self.cap, out=self.lay, recv_x=self.recv_x, recv_scale=self.recv_scale,
-                    workspace=self.ws, status=self.status), b["layout"] + b["dispatch_fp8"]))
+                    workspace=self.ws, status=self.status, pow2_scales=self.pow2), b["layout"] + b["dispatch_fp8"]))
         else:
             calls.append(("dispatch_bf16", lambda: cgl.dispatch_bf16(self.x, dst, rows, recv_x=self.recv_x,
                                                                      status=self.status), b["dispatch_bf16"]))
@@ -577,7 +580,8 @@ def run_e2e(step: GpuStep, steps: int):
 
 # ----------------------------------------------------------------- CPU oracle timing
 
-def oracle_step_seconds(inp: W.Inputs, y: np.ndarray, tokens: int, reps_min_s: float, max_reps: int):
+def oracle_step_seconds(inp: W.Inputs, y: np.ndarray, tokens: int, reps_min_s: float, max_reps: int,
+                        pow2: bool = False):
     """Time the oracle's layout + dispatch + combine on the first `tokens` tokens."""
     import oracle
 
@@ -591,7 +595,7 @@ def oracle_step_seconds(inp: W.Inputs, y: np.ndarray, tokens: int, reps_min_s: f
         L = oracle.get_layout(idx, wl.num_experts, wl.num_ranks, 0)
         rows = idx.size
         if wl.fp8:
-            oracle.dispatch_fp8(x, L.dst_pos, rows)
+            oracle.dispatch_fp8(x, L.dst_pos, rows, pow2_scales=pow2)
         else:
             oracle.dispatch_bf16(x, L.dst_pos, rows)
         oracle.combine(y[:rows], L.dst_pos, w)
@@ -626,7 +630,8 @@ def base_line(args, wl, n_gpus):
         "dtype": ("f32 arithmetic; bf16 x in, e4m3 + f32 scale rows out, bf16 combine" if wl.fp8
                   else "f32 arithmetic; bf16 rows"), "data": "synthetic",
         "config": {
-            "workload": workload_label(wl, getattr(args, "dedup", False)), "num_tokens": wl.num_tokens, "hidden": wl.hidden,
+            "workload": workload_label(wl, getattr(args, "dedup", False), getattr(args, "ue8m0", False)),
+            "num_tokens": wl.num_tokens, "hidden": wl.hidden,
             "num_experts": wl.num_experts, "num_groups": wl.num_groups, "topk_group": wl.topk_group,
             "topk": wl.topk, "num_ranks": wl.num_ranks,
             "storage": ("x bf16 -> e4m3 rows + f32 1x128 scales; combine bf16 in, f32 accumulate, bf16 out"
@@ -650,14 +655,14 @@ def run_reference(args):
     y = W.expert_outputs(inp.topk_idx.size, wl.hidden, args.seed)
     threads = oracle.set_threads(cpu_threads())
     # size the per-step sample so that warmup + steps end within ~2 minutes
-    t_full, _ = oracle_step_seconds(inp, y, wl.num_tokens, 0.0, 1)
+    t_full, _ = oracle_step_seconds(inp, y, wl.num_tokens, 0.0, 1, args.ue8m0)
     budget = 120.0 / max(1, args.steps + args.warmup)
     tokens = wl.num_tokens if t_full <= budget else max(16, int(wl.num_tokens * budget / t_full) // 16 * 16)
     for _ in range(args.warmup):
-        oracle_step_seconds(inp, y, tokens, 0.0, 1)
+        oracle_step_seconds(inp, y, tokens, 0.0, 1, args.ue8m0)
     times = []
     for _ in range(args.steps):
-        t, _ = oracle_step_seconds(inp, y, tokens, 0.0, 1)
+        t, _ = oracle_step_seconds(inp, y, tokens, 0.0, 1, args.ue8m0)
         times.append(t)
     sec = sum(times) / len(times)
     gbs = step_bytes_for(wl, tokens) / sec / 1e9
@@ -689,7 +694,7 @@ def run_ours(args):
 
         wl = dataclasses.replace(wl, num_tokens=args.num_tokens)
     step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup, full_backward=args.full_backward,
-                   fused_decode=args.fused_decode, split_layout=args.split_layout)
+                   fused_decode=args.fused_decode, split_layout=args.split_layout, pow2_scales=args.ue8m0)
     phases = step.kernels()
 
     graph = None if args.no_graph else capture_step(step)
@@ -810,7 +815,7 @@ def run_ours(args):
         import oracle
 
         threads = oracle.set_threads(cpu_threads())
-        t, reps = oracle_step_seconds(step.host, step.host_y, wl.num_tokens, args.cpu_seconds, 1000)
+        t, reps = oracle_step_seconds(step.host, step.host_y, wl.num_tokens, args.cpu_seconds, 1000, args.ue8m0)
         gbs = step_bytes_for(wl, wl.num_tokens) * reps / t / 1e9
         line["cpu_baseline"] = {
             "value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -844,6 +849,7 @@ def main(argv=None):
     ap.add_argument("--split-layout", action="store_true",
                     help="FP8: cgl_get_layout and cgl_dispatch_fp8 as two calls instead of cgl_layout_dispatch_fp8")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--ue8m0", action="store_true", help="FP8: power-of-two (UE8M0) scales instead of amax / 448")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

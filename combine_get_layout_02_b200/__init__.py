@@ -48,7 +48,10 @@ class CglError(RuntimeError):
 
 
 class Opts(C.Structure):
-    _fields_ = [("num_sms", C.c_int32), ("capacity", C.c_int32)]
+    _fields_ = [("num_sms", C.c_int32), ("capacity", C.c_int32), ("flags", C.c_uint32)]
+
+
+OPT_UE8M0_SCALES = 1   # cgl_opts.flags: power-of-two (UE8M0) FP8 scales
 
 
 _lib = None
@@ -131,8 +134,8 @@ def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None):
     return t
 
 
-def _opts(num_sms: int = 0, capacity: int = 0):
-    return C.byref(Opts(int(num_sms), int(capacity)))
+def _opts(num_sms: int = 0, capacity: int = 0, pow2_scales: bool = False):
+    return C.byref(Opts(int(num_sms), int(capacity), OPT_UE8M0_SCALES if pow2_scales else 0))
 
 
 def new_status(device=None) -> torch.Tensor:
@@ -249,9 +252,10 @@ def get_rank_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, ca
 
 def dispatch_fp8(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
                  recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
-                 status: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None):
+                 status: Optional[torch.Tensor] = None, num_sms: int = 0, pow2_scales: bool = False, stream=None):
     """FP8 E4M3 dispatch with per-token 1x128 fp32 scales (cgl_dispatch_fp8).
 
+    pow2_scales: power-of-two (UE8M0) scales (CGL_OPT_UE8M0_SCALES).
     Returns (recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128]); rows that
     receive no copy are left as they were (uninitialised when allocated here)."""
     x = _dev(x, "x", torch.bfloat16, 2)
@@ -263,7 +267,7 @@ def dispatch_fp8(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
     if recv_scale is None:
         recv_scale = torch.empty((num_recv_rows, h // 128), dtype=torch.float32, device=x.device)
     code = lib().cgl_dispatch_fp8(_ptr(x), n, h, k, _ptr(dst), _ptr(recv_x), _ptr(recv_scale),
-                                  int(num_recv_rows), _opts(num_sms), _ptr(status), _stream(stream))
+                                  int(num_recv_rows), _opts(num_sms, 0, pow2_scales), _ptr(status), _stream(stream))
     _check(code, "cgl_dispatch_fp8")
     return recv_x, recv_scale
 
@@ -326,7 +330,8 @@ def combine_backward(grad_out: torch.Tensor, y: torch.Tensor, dst_pos: torch.Ten
 def decode_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: int, num_ranks: int,
                         capacity: int = 0, *, out: Optional[Layout] = None,
                         recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
-                        status: Optional[torch.Tensor] = None, num_sms: int = 0, stream=None):
+                        status: Optional[torch.Tensor] = None, num_sms: int = 0, pow2_scales: bool = False,
+                        stream=None):
     """Layout + FP8 dispatch of a small (decode) batch in one launch (cgl_decode_dispatch_fp8).
 
     Returns (Layout, recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128])."""
@@ -352,7 +357,7 @@ def decode_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: in
     if recv_scale is None:
         recv_scale = torch.empty((rows, h // 128), dtype=torch.float32, device=dev)
     code = lib().cgl_decode_dispatch_fp8(
-        _ptr(idx), n, k, E, R, _opts(num_sms, capacity), _ptr(x), h, _ptr(out.tokens_per_expert),
+        _ptr(idx), n, k, E, R, _opts(num_sms, capacity, pow2_scales), _ptr(x), h, _ptr(out.tokens_per_expert),
         _ptr(out.tokens_per_rank), _ptr(out.is_token_in_rank), _ptr(out.expert_offset), _ptr(out.max_count),
         _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(recv_x), _ptr(recv_scale), _ptr(status), _stream(stream))
     _check(code, "cgl_decode_dispatch_fp8")
@@ -373,7 +378,7 @@ def layout_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: in
                         capacity: int = 0, *, out: Optional[Layout] = None,
                         recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
-                        num_sms: int = 0, stream=None):
+                        num_sms: int = 0, pow2_scales: bool = False, stream=None):
     """Layout + FP8 dispatch of any batch in one call (cgl_layout_dispatch_fp8).
 
     Returns (Layout, recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128])."""
@@ -404,7 +409,7 @@ def layout_dispatch_fp8(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: in
     if recv_scale is None:
         recv_scale = torch.empty((rows, h // 128), dtype=torch.float32, device=dev)
     code = lib().cgl_layout_dispatch_fp8(
-        _ptr(idx), n, k, E, R, _opts(num_sms, capacity), _ptr(x), h, _ptr(out.tokens_per_expert),
+        _ptr(idx), n, k, E, R, _opts(num_sms, capacity, pow2_scales), _ptr(x), h, _ptr(out.tokens_per_expert),
         _ptr(out.tokens_per_rank), _ptr(out.is_token_in_rank), _ptr(out.expert_offset), _ptr(out.max_count),
         _ptr(out.dst_pos), _ptr(out.recv_src), _ptr(recv_x), _ptr(recv_scale), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))

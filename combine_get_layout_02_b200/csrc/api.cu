@@ -32,6 +32,9 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int opt_sms(const cgl_opts *o) { return o ? o->num_sms : 0; }
 int opt_cap(const cgl_opts *o) { return o ? o->capacity : 0; }
+uint32_t opt_flags(const cgl_opts *o) { return o ? o->flags : 0u; }
+bool flags_ok(const cgl_opts *o) { return (opt_flags(o) & ~CGL_OPT_UE8M0_SCALES) == 0; }
+bool opt_pow2(const cgl_opts *o) { return (opt_flags(o) & CGL_OPT_UE8M0_SCALES) != 0; }
 
 }  // namespace
 
@@ -125,7 +128,7 @@ using namespace cgl;
 
 extern "C" {
 
-int cgl_version(void) { return 100; }
+int cgl_version(void) { return 200; }
 
 const char *cgl_status_string(int s) {
     switch (s) {
@@ -161,7 +164,7 @@ cgl_status cgl_get_layout(const int32_t *topk_idx, int64_t n, int k, int E, int 
                           uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
                           int32_t *dst_pos, int32_t *recv_src, void *workspace,
                           size_t workspace_bytes, uint32_t *status_dev, void *stream) {
-    if (!layout_sizes_ok(n, k, E, R)) return CGL_EINVAL;
+    if (!layout_sizes_ok(n, k, E, R) || !flags_ok(opts)) return CGL_EINVAL;
     const int cap = opt_cap(opts);
     if (cap < 0 || (int64_t)E * cap >= ((int64_t)1 << 31)) return CGL_EINVAL;
     const int64_t rows = cap > 0 ? (int64_t)E * cap : n * k;
@@ -185,7 +188,7 @@ cgl_status cgl_get_rank_layout(const int32_t *topk_idx, int64_t n, int k, int E,
                                int32_t *max_count, int32_t *rank_dst, int32_t *recv_token,
                                void *workspace, size_t workspace_bytes, uint32_t *status_dev,
                                void *stream) {
-    if (!layout_sizes_ok(n, k, E, R)) return CGL_EINVAL;
+    if (!layout_sizes_ok(n, k, E, R) || !flags_ok(opts)) return CGL_EINVAL;
     const int cap = opt_cap(opts);
     if (cap < 0 || (int64_t)R * cap >= ((int64_t)1 << 31)) return CGL_EINVAL;
     const int64_t rows = cap > 0 ? (int64_t)R * cap : n * k;
@@ -207,13 +210,13 @@ cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const in
                             const cgl_opts *opts, uint32_t *status_dev, void *stream) {
     if (n < 0 || h <= 0 || h % 128 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0)
         return CGL_EINVAL;
-    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0 || !flags_ok(opts)) return CGL_EINVAL;
     if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && (!recv_x || !recv_scale)) return CGL_EINVAL;
     if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) ||
         !aligned(recv_scale, 4) || !aligned(status_dev, 4))
         return CGL_EALIGN;
-    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, opt_sms(opts),
+    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, opt_sms(opts), opt_pow2(opts),
                                status_dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -221,7 +224,7 @@ cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const i
                              uint16_t *recv_x, int64_t recv_rows, const cgl_opts *opts,
                              uint32_t *status_dev, void *stream) {
     if (n < 0 || h <= 0 || h % 8 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0) return CGL_EINVAL;
-    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0 || !flags_ok(opts)) return CGL_EINVAL;
     if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && !recv_x) return CGL_EINVAL;
     if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) || !aligned(status_dev, 4))
@@ -234,7 +237,7 @@ cgl_status cgl_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_
                        const float *topk_weights, int64_t n, int h, int k, uint16_t *out,
                        const cgl_opts *opts, uint32_t *status_dev, void *stream) {
     if (n < 0 || h <= 0 || h % 8 != 0 || k < 1 || k > kMaxTopk || recv_rows < 0) return CGL_EINVAL;
-    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0 || !flags_ok(opts)) return CGL_EINVAL;
     if (n > 0 && (!dst_pos || !topk_weights || !out)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && !y) return CGL_EINVAL;
     if (!aligned(y, 16) || !aligned(out, 16) || !aligned(dst_pos, 4) ||
@@ -250,7 +253,7 @@ cgl_status cgl_combine_backward(const uint16_t *grad_out, const uint16_t *y, int
                                 uint32_t *status_dev, void *stream) {
     if (n < 0 || h <= 0 || h % 16 != 0 || h > 16384 || k < 1 || k > kMaxTopk || recv_rows < 0)
         return CGL_EINVAL;
-    if (opt_sms(opts) < 0) return CGL_EINVAL;
+    if (opt_sms(opts) < 0 || !flags_ok(opts)) return CGL_EINVAL;
     if (n > 0 && (!grad_out || !dst_pos || !topk_weights || !grad_w)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && (!y || !grad_y)) return CGL_EINVAL;
     if (!aligned(grad_out, 16) || !aligned(y, 16) || !aligned(grad_y, 16) || !aligned(dst_pos, 4) ||
@@ -266,7 +269,7 @@ cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
                                    uint8_t *is_token_in_rank, int32_t *expert_offset, int32_t *max_count,
                                    int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
                                    float *recv_scale, uint32_t *status_dev, void *stream) {
-    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0) return CGL_EINVAL;
+    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0 || !flags_ok(opts)) return CGL_EINVAL;
     const int per_block = 1024 / k < 256 ? 1024 / k : 256;   // tokens one layout block holds
     if (n > per_block) return CGL_EINVAL;
     if (decode_fused_smem_bytes(n, k, E, R) > 47 * 1024) return CGL_EINVAL;
@@ -283,7 +286,8 @@ cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
         return CGL_EALIGN;
     return launch_decode_dispatch_fp8(topk_idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank,
                                       is_token_in_rank, expert_offset, max_count, dst_pos, recv_src, recv_x,
-                                      recv_scale, opt_sms(opts), status_dev, static_cast<cudaStream_t>(stream));
+                                      recv_scale, opt_sms(opts), opt_pow2(opts), status_dev,
+                                      static_cast<cudaStream_t>(stream));
 }
 
 size_t cgl_layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
@@ -304,7 +308,7 @@ cgl_status cgl_layout_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
                                    int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x, float *recv_scale,
                                    void *workspace, size_t workspace_bytes, uint32_t *status_dev,
                                    void *stream) {
-    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0) return CGL_EINVAL;
+    if (!layout_sizes_ok(n, k, E, R) || h <= 0 || h % 128 != 0 || !flags_ok(opts)) return CGL_EINVAL;
     const int cap = opt_cap(opts);
     if (cap < 0 || (int64_t)E * cap >= ((int64_t)1 << 31) || opt_sms(opts) < 0) return CGL_EINVAL;
     const int64_t rows = cap > 0 ? (int64_t)E * cap : n * k;
@@ -320,7 +324,7 @@ cgl_status cgl_layout_dispatch_fp8(const int32_t *topk_idx, int64_t n, int k, in
         return CGL_EALIGN;
     return launch_layout_dispatch_fp8(topk_idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank,
                                       is_token_in_rank, expert_offset, max_count, dst_pos, recv_src, recv_x,
-                                      recv_scale, workspace, opt_sms(opts), status_dev,
+                                      recv_scale, workspace, opt_sms(opts), opt_pow2(opts), status_dev,
                                       static_cast<cudaStream_t>(stream));
 }
 

@@ -100,6 +100,31 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// 2^e as a float, for e in [-126, 127].
+__device__ __forceinline__ float exp2_int(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// The block's scale and reciprocal.  IEEE: scale = amax_c / 448, inv = 448 /
+// amax_c (correctly rounded divisions).  Power of two (UE8M0): scale = 2^e for
+// the smallest integer e with 448 * 2^e >= amax_c, inv = 2^-e.  e starts from
+// the exponent of the rounded quotient amax_c / 448, rounded up unless that
+// quotient is a power of two; the rounding can leave it one off on either side
+// of a power of two, so two comparisons of 448 * 2^e (exact in binary32) with
+// amax_c settle it.  amax_c in [1e-4, FLT_MAX] keeps e in [-22, 120].
+__device__ __forceinline__ void block_scale(float amax_c, bool pow2, float &scale, float &inv) {
+    if (!pow2) {
+        scale = __fdiv_rn(amax_c, 448.0f);
+        inv = __fdiv_rn(448.0f, amax_c);
+        return;
+    }
+    const uint32_t s = __float_as_uint(__fdiv_rn(amax_c, 448.0f));
+    int e = (int)((s >> 23) & 0xFFu) - 127;
+    if (s & 0x7FFFFFu) ++e;
+    if (__fmul_rn(448.0f, exp2_int(e - 1)) >= amax_c) --e;
+    if (__fmul_rn(448.0f, exp2_int(e)) < amax_c) ++e;
+    scale = exp2_int(e);
+    inv = exp2_int(-e);
+}
+
 // Widen the low / high BF16 of a 32-bit word to float (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

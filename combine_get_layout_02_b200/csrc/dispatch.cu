@@ -5,6 +5,8 @@
 // normal kernels (news article "具体性能方面", brainleap "DeepEP 的性能表现",
 // flashmla.org/de); "原生FP8 调度支持" is item 5 of brainleap's key techniques.
 // The kernels here copy inside one GPU's HBM instead of over NVLink/RDMA.
+// The scale is amax_c / 448 by IEEE division, or with `pow2` the smallest
+// power of two 2^e with 448 * 2^e >= amax_c (block_scale in common.cuh).
 //
 // FP8, hidden <= 16384 (the bulk kernel).  A CTA owns one token at a time
 // (persistent over tokens), one thread per 16 hidden values: the thread loads
@@ -37,7 +39,7 @@ constexpr int kMaxBulkHiddenBf16 = 8192; // two staged BF16 rows stay within 32 
 __global__ void __launch_bounds__(1024)
 dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                          const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
-                         float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
+                         float *__restrict__ recv_scale, int64_t recv_rows, int pow2, uint32_t *status) {
     extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][h] staged code rows
     griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4, nblk = h >> 7;
@@ -64,8 +66,8 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
         const float amax_c = fmaxf(m, 1e-4f);
-        const float scale = __fdiv_rn(amax_c, 448.0f);
-        const float inv = __fdiv_rn(448.0f, amax_c);
+        float scale, inv;
+        block_scale(amax_c, pow2 != 0, scale, inv);
         const uint4 q = quant16(a, b, inv);
         uint8_t *row = rows_smem + buf * h;
         if (threadIdx.x == 0) bulk_wait_read<1>();   // copies from two tokens ago have read `row`
@@ -99,7 +101,7 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
 __global__ void __launch_bounds__(kThreads)
 dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                     const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
-                    float *__restrict__ recv_scale, int64_t recv_rows, uint32_t *status) {
+                    float *__restrict__ recv_scale, int64_t recv_rows, int pow2, uint32_t *status) {
     griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4;        // 16 values per thread
     const int nblk = h >> 7;          // 128-value scale blocks per row
@@ -137,8 +139,8 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
         if (!active) continue;
         const float amax_c = fmaxf(m, 1e-4f);
-        const float scale = __fdiv_rn(amax_c, 448.0f);
-        const float inv = __fdiv_rn(448.0f, amax_c);
+        float scale, inv;
+        block_scale(amax_c, pow2 != 0, scale, inv);
         uint32_t qw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -240,7 +242,7 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
 
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
-                               int num_sms, uint32_t *status, cudaStream_t stream) {
+                               int num_sms, bool pow2, uint32_t *status, cudaStream_t stream) {
     if (n * (h / 16) == 0) return CGL_OK;
     if (h <= kMaxBulkHidden) {
         const int threads = (h / 16 + 31) / 32 * 32;
@@ -249,7 +251,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
         if (grid <= 0) return CGL_ECUDA;
         const cudaError_t err = launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)2 * h, stream, x, n, h, k, dst_pos, recv_x,
-                                           recv_scale, recv_rows, status);
+                                           recv_scale, recv_rows, (int)pow2, status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
     }
     const int64_t work = n * (h / 16);
@@ -257,7 +259,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
                                (work + kThreads - 1) / kThreads, num_sms);
     if (grid <= 0) return CGL_ECUDA;
     const cudaError_t err = launch_pdl(dispatch_fp8_kernel, dim3(grid), dim3(kThreads), 0, stream, x, n, h,
-                                       k, dst_pos, recv_x, recv_scale, recv_rows, status);
+                                       k, dst_pos, recv_x, recv_scale, recv_rows, (int)pow2, status);
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 

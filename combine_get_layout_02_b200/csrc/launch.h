@@ -63,9 +63,10 @@ cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R
                               int32_t *rank_dst, int32_t *recv_token, void *ws, uint32_t *status,
                               cudaStream_t stream);
 
+// pow2: power-of-two (UE8M0) scales instead of amax_c / 448 (cgl_opts.flags).
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
-                               int num_sms, uint32_t *status, cudaStream_t stream);
+                               int num_sms, bool pow2, uint32_t *status, cudaStream_t stream);
 
 cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                 uint16_t *recv_x, int64_t recv_rows, int num_sms, uint32_t *status,
@@ -86,8 +87,8 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       const uint16_t *x, int h, int32_t *tokens_per_expert,
                                       int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
                                       int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
-                                      uint8_t *recv_x, float *recv_scale, int num_sms, uint32_t *status,
-                                      cudaStream_t stream);
+                                      uint8_t *recv_x, float *recv_scale, int num_sms, bool pow2,
+                                      uint32_t *status, cudaStream_t stream);
 
 // Fused layout + FP8 dispatch (one cooperative launch when it applies, else
 // the layout and the dispatch kernels in turn).
@@ -97,7 +98,7 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       const uint16_t *x, int h, int32_t *tokens_per_expert,
                                       int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
                                       int32_t *max_count, int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
-                                      float *recv_scale, void *ws, int num_sms, uint32_t *status,
+                                      float *recv_scale, void *ws, int num_sms, bool pow2, uint32_t *status,
                                       cudaStream_t stream);
 
 cgl_status launch_combine_backward(const uint16_t *g, const uint16_t *y, int64_t recv_rows,

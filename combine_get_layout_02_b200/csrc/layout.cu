@@ -1175,7 +1175,7 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
                     int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
                     int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
                     int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
-                    uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, uint32_t *status) {
+                    uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, int pow2, uint32_t *status) {
     extern __shared__ __align__(16) int32_t smem_decode[];
     __shared__ int32_t scan_tmp[32];
     const Smem s = carve_rep(smem_decode, T, E, R);
@@ -1205,8 +1205,8 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
         if (!active) continue;
         const float amax_c = fmaxf(m, 1e-4f);
-        const float scale = __fdiv_rn(amax_c, 448.0f);
-        const float inv = __fdiv_rn(448.0f, amax_c);
+        float scale, inv;
+        block_scale(amax_c, pow2 != 0, scale, inv);
         const uint4 q = quant16(a, b, inv);
         for (int j = 0; j < k; ++j) {
             const int32_t row = s_dst[tl * k + j];
@@ -1306,7 +1306,8 @@ __device__ __forceinline__ void stage_load(const uint16_t *__restrict__ x, int h
     }
 }
 
-__device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch &B, uint8_t *qbuf, float *sbuf) {
+__device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch &B, uint8_t *qbuf, float *sbuf,
+                                               int pow2) {
     const int nblk = h >> 7;
 #pragma unroll
     for (int u = 0; u < kStageUnroll; ++u) {
@@ -1317,8 +1318,8 @@ __device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch 
         for (int o = kStageLanes / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         if (B.t[u] < cnt) {
             const float amax_c = fmaxf(m, 1e-4f);
-            const float scale = __fdiv_rn(amax_c, 448.0f);
-            const float inv = __fdiv_rn(448.0f, amax_c);
+            float scale, inv;
+            block_scale(amax_c, pow2 != 0, scale, inv);
             uint4 *dst = reinterpret_cast<uint4 *>(qbuf + (size_t)B.t[u] * h + (size_t)B.c[u] * kStageV);
 #pragma unroll
             for (int i = 0; i < kStageLoads; i += 2) dst[i / 2] = quant16(B.d[u][i], B.d[u][i + 1], inv);
@@ -1337,7 +1338,7 @@ __device__ __forceinline__ void stage_quantise(int h, int cnt, const StageBatch 
 // it at the end: every calling warp arrives on every group exactly once.
 __device__ void stage_fp8_rows_grouped(const uint16_t *__restrict__ x, int h, int64_t t_first, int cnt,
                                        int tok_begin, int tok_end, uint8_t *qbuf, float *sbuf, int th0, int nth,
-                                       int ng, int bar_count) {
+                                       int ng, int bar_count, int pow2) {
     const int chunks = h / kStageV;    // a multiple of kStageLanes: a scale block never straddles tokens
     const int q0 = tok_begin * chunks, q1 = tok_end * chunks;
     const int me = (int)threadIdx.x - th0;
@@ -1362,13 +1363,13 @@ __device__ void stage_fp8_rows_grouped(const uint16_t *__restrict__ x, int h, in
     for (int base = q0; base < q1;) {
         const bool has1 = base + step < q1;
         if (has1) stage_load(x, h, t_first, tok_end, chunks, dt, dc, t, c, b1);
-        stage_quantise(h, tok_end, b0, qbuf, sbuf);
+        stage_quantise(h, tok_end, b0, qbuf, sbuf, pow2);
         base += step;
         arrive_below((int64_t)wme + base);
         if (!has1) break;
         const bool has2 = base + step < q1;
         if (has2) stage_load(x, h, t_first, tok_end, chunks, dt, dc, t, c, b0);
-        stage_quantise(h, tok_end, b1, qbuf, sbuf);
+        stage_quantise(h, tok_end, b1, qbuf, sbuf, pow2);
         base += step;
         arrive_below((int64_t)wme + base);
         if (!has2) break;
@@ -1408,7 +1409,7 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
                            int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
                            int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
                            const uint16_t *__restrict__ x, int h, uint8_t *__restrict__ recv_x,
-                           float *__restrict__ recv_scale, int scale_bulk, uint32_t *status) {
+                           float *__restrict__ recv_scale, int scale_bulk, int pow2, uint32_t *status) {
     extern __shared__ __align__(128) int32_t smem_ld[];
     __shared__ int32_t scan_tmp[32];
     const Smem s = carve_rep(smem_ld, T, E, R);
@@ -1448,10 +1449,11 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
             }
             bulk_wait_all();
         } else {   // warps 1-7, free after the layout: the CTA's last tokens
-            stage_fp8_rows_grouped(x, h, t0, cnt0, split, cnt0, qbuf, sbuf, 32, kThreads - 32, ng, kLdThreads);
+            stage_fp8_rows_grouped(x, h, t0, cnt0, split, cnt0, qbuf, sbuf, 32, kThreads - 32, ng, kLdThreads, pow2);
         }
     } else {
-        stage_fp8_rows_grouped(x, h, t0, cnt0, 0, split, qbuf, sbuf, kThreads, kLdThreads - kThreads, ng, kLdThreads);
+        stage_fp8_rows_grouped(x, h, t0, cnt0, 0, split, qbuf, sbuf, kThreads, kLdThreads - kThreads, ng, kLdThreads,
+                               pow2);
     }
 }
 
@@ -1652,14 +1654,15 @@ template <int CH>
 cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, int E, int R, int cap,
                      const uint16_t *x, int h, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
                      uint8_t *in_rank, int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
-                     int32_t *recv_src, uint8_t *recv_x, float *recv_scale, uint32_t *status, cudaStream_t stream) {
+                     int32_t *recv_src, uint8_t *recv_x, float *recv_scale, bool pow2, uint32_t *status,
+                     cudaStream_t stream) {
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
     const int scale_bulk = ((h >> 7) % 4 == 0) && (reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0);
     const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
     const cudaError_t err = launch_pdl(layout_dispatch_fp8_kernel<CH>, dim3((unsigned)sh.G), dim3(kLdThreads), sh.smem,
                                        stream, idx, n, k, E, R, cap, sh.T, sh.B, vec, tokens_per_expert,
                                        tokens_per_rank, in_rank, expert_offset, max_count, dst_pos, recv_src,
-                                       recv_rows, x, h, recv_x, recv_scale, scale_bulk, status);
+                                       recv_rows, x, h, recv_x, recv_scale, scale_bulk, (int)pow2, status);
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }
 
@@ -1679,27 +1682,30 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       const uint16_t *x, int h, int32_t *tokens_per_expert,
                                       int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
                                       int32_t *max_count, int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
-                                      float *recv_scale, void *ws, int num_sms, uint32_t *status,
+                                      float *recv_scale, void *ws, int num_sms, bool pow2, uint32_t *status,
                                       cudaStream_t stream) {
     const LdShape sh = ld_shape(n, k, E, R, h, num_sms);
     if (ld_fits(sh)) {
         switch (sh.CH) {
             case 1:
                 return ld_launch<1>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, pow2, status,
+                                    stream);
             case 2:
                 return ld_launch<2>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, pow2, status,
+                                    stream);
             default:
                 return ld_launch<4>(sh, idx, n, k, E, R, cap, x, h, tokens_per_expert, tokens_per_rank, in_rank,
-                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, status, stream);
+                                    expert_offset, max_count, dst_pos, recv_src, recv_x, recv_scale, pow2, status,
+                                    stream);
         }
     }
     const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
                                         expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
     if (st != CGL_OK) return st;
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
-    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, num_sms, status, stream);
+    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, num_sms, pow2, status, stream);
 }
 
 bool layout_needs_smem_optin(int E, int R, int k) {
@@ -1870,7 +1876,7 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       const uint16_t *x, int h, int32_t *tokens_per_expert,
                                       int32_t *tokens_per_rank, uint8_t *in_rank, int32_t *expert_offset,
                                       int32_t *max_count, int32_t *dst_pos, int32_t *recv_src,
-                                      uint8_t *recv_x, float *recv_scale, int num_sms, uint32_t *status,
+                                      uint8_t *recv_x, float *recv_scale, int num_sms, bool pow2, uint32_t *status,
                                       cudaStream_t stream) {
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
     const int sms = device_sm_count();
@@ -1884,17 +1890,17 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
         case 1:
             err = launch_pdl(decode_fused_kernel<1>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
                              R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
             break;
         case 2:
             err = launch_pdl(decode_fused_kernel<2>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
                              R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
             break;
         default:
             err = launch_pdl(decode_fused_kernel<4>, dim3((unsigned)d.G), dim3(kThreads), smem, stream, idx, n, k, E,
                              R, cap, d.T, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, status);
+                             max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
     }
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
 }

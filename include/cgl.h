@@ -78,9 +78,22 @@ typedef struct cgl_opts {
      * the decode setting pads to the largest per-expert count, which the host
      * reads from a first, compact call (max_count). */
     int32_t capacity;
+    /* Bit flags (0 = none; bits this library does not define are refused with
+     * CGL_EINVAL).  CGL_OPT_UE8M0_SCALES: the FP8 dispatch calls
+     * (cgl_dispatch_fp8, cgl_layout_dispatch_fp8, cgl_decode_dispatch_fp8) use
+     * power-of-two scales, as an 8-bit exponent-only (UE8M0) scale format holds:
+     * per 128-value block, scale = 2^e for the smallest integer e with
+     * 448 * 2^e >= amax_c, inv = 2^-e, codes = e4m3_rn_satfinite(x * inv) (x * inv
+     * is exact, and no value saturates).  recv_scale still holds binary32
+     * values: 2^e, whose biased exponent field ((bits >> 23) & 0xFF) is the
+     * UE8M0 code.  Calls that quantise nothing ignore the flag. */
+    uint32_t flags;
 } cgl_opts;
 
-/* Library version (major * 10000 + minor * 100 + patch). */
+#define CGL_OPT_UE8M0_SCALES 1u
+
+/* Library version (major * 10000 + minor * 100 + patch).  0.2.0 added
+ * cgl_opts.flags: C callers built against an older cgl.h must be rebuilt. */
 int cgl_version(void);
 
 /* A static string naming a cgl_status value (or "unknown status"). */
@@ -225,7 +238,8 @@ cgl_status cgl_get_layout_noalloc(const int32_t *topk_idx, int64_t num_tokens, i
  *
  * For token t and each block b of 128 consecutive hidden values:
  *   amax = max |x|, amax_c = max(amax, 1e-4), scale = amax_c / 448,
- *   inv = 448 / amax_c (IEEE binary32 divisions), q = e4m3_rn_satfinite(x * inv);
+ *   inv = 448 / amax_c (IEEE binary32 divisions), q = e4m3_rn_satfinite(x * inv)
+ *   (with CGL_OPT_UE8M0_SCALES: scale = 2^e, inv = 2^-e, see cgl_opts.flags);
  * then for every slot j with dst_pos[t, j] = row >= 0:
  *   recv_x[row, :] = q, recv_scale[row, b] = scale.
  * In (device): x BF16 [num_tokens, hidden]; dst_pos int32 [num_tokens, num_topk]

@@ -213,3 +213,26 @@ def test_noalloc_limits_at_their_exact_boundaries(L):
     # k = 8, R = 32: T = 128 tokens per block, 12 E + 32 + 128 <= 9984 -> E <= 818 (800 and 832 are multiples of 32)
     assert call(1000, 8, 800, 32) in accepted
     assert call(1000, 8, 832, 32) == cgl.EINVAL
+
+
+def test_opts_flags_unknown_bits_refused(L):
+    """cgl_opts.flags: CGL_OPT_UE8M0_SCALES is the only defined bit; any other bit is
+    refused with CGL_EINVAL before anything is launched (fake pointers never used)."""
+    src = open(os.path.join(ROOT, "include", "cgl.h")).read()
+    assert "#define CGL_OPT_UE8M0_SCALES 1u" in src and "uint32_t flags;" in src
+    assert L.cgl_version() >= 200
+    p = FAKE
+    bad = C.byref(cgl.Opts(0, 0, 2))
+    assert L.cgl_dispatch_fp8(p, 128, 7168, 8, p, p, p, 1024, bad, p, None) == cgl.EINVAL
+    assert L.cgl_dispatch_bf16(p, 128, 7168, 8, p, p, 1024, bad, p, None) == cgl.EINVAL
+    assert L.cgl_combine(p, 1024, p, p, 128, 7168, 8, p, bad, p, None) == cgl.EINVAL
+    ws = L.cgl_layout_workspace_bytes(128, 8, 256, 64)
+    assert L.cgl_get_layout(p, 128, 8, 256, 64, bad, p, p, p, p, p, p, p, p, ws, p, None) == cgl.EINVAL
+    assert L.cgl_decode_dispatch_fp8(p, 128, 8, 256, 32, bad, p, 7168, p, p, p, p, p, p, p, p, p, p, None) \
+        == cgl.EINVAL
+    wsd = L.cgl_layout_dispatch_workspace_bytes(4096, 8, 256, 64)
+    assert L.cgl_layout_dispatch_fp8(p, 4096, 8, 256, 64, bad, p, 7168, p, p, p, p, p, p, p, p, p, p, wsd, p,
+                                     None) == cgl.EINVAL
+    # the defined bit passes the flag check (then fails on a misaligned pointer, as without it)
+    ok = C.byref(cgl.Opts(0, 0, cgl.OPT_UE8M0_SCALES))
+    assert L.cgl_dispatch_fp8(p + 8, 128, 7168, 8, p, p, p, 1024, ok, p, None) == cgl.EALIGN
