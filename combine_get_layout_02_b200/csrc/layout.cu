@@ -1217,6 +1217,202 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     }
 }
 
+// Decode batches of at most one token per SM: one CTA per token.  CTA t
+// needs, for its own k copies, the copies of each expert in tokens before t
+// and the expert offsets; everything else is the block's share of the global
+// outputs.  Each of the first n threads reads one token's ids (one round of
+// loads) and counts them into before[] / rest[] (shared reductions), the
+// batch's valid ids, and distinct tokens of the CTA's designated ranks (t, t +
+// n, ...: one ballot per rank).  Then each own slot j is ranked by one warp:
+// offset = the sum of totals below its expert (a warp reduction, so no block
+// scan outside CTA 0), rank = before[e] + the earlier slots of the token with
+// that expert.  CTA 0 writes the expert counts, offsets and max; every CTA
+// writes its token's rows, is_token_in_rank row and share of the recv_src
+// fill, then quantises the token as the fused decode kernel does.  About five
+// block barriers where the general block takes a dozen.
+template <int KM>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int vec,
+                    const uint16_t *__restrict__ x, int h, int32_t *__restrict__ tokens_per_expert,
+                    int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
+                    int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
+                    int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
+                    uint8_t *__restrict__ recv_x, float *__restrict__ recv_scale, int pow2, uint32_t *status) {
+    __shared__ int32_t s_before[kMaxExperts];   // copies in tokens before this CTA's
+    __shared__ int32_t s_total[kMaxExperts];    // copies in the rest, then in all tokens
+    __shared__ int32_t s_off[kMaxExperts];      // CTA 0: exclusive prefix of s_total
+    __shared__ int32_t s_own[kMaxTopk];         // this token's ids
+    __shared__ int32_t s_row[kMaxTopk];         // their receive rows
+    __shared__ uint32_t s_mask[32];             // this token's rank set (R <= 1024)
+    __shared__ int32_t s_cnt[1 + 32];           // [0]: valid ids of the batch; [1 + i]: designated rank i
+    __shared__ int32_t scan_tmp[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x, b = blockIdx.x;
+    const int64_t t = b;
+    const bool has_tok = t < n;
+    const int nd = G > 1 ? rep_designated(b, G, R) : 0;
+    const uint32_t rm = div_magic(E / R), gm = div_magic(G);
+    griddep_wait();   // ids and x may come from the kernels just before
+    // this thread's token (n <= 256 = the block size): its ids, in flight while zeroing
+    int32_t ids[KM];
+    const int64_t tp = tid;
+    {
+        const int32_t *src = idx + tp * k;
+        if (vec) {
+#pragma unroll
+            for (int q = 0; q < KM / 4; ++q) {
+                int4 v = make_int4(-1, -1, -1, -1);
+                if (tp < n && q * 4 < k) v = __ldg(reinterpret_cast<const int4 *>(src) + q);
+                ids[4 * q] = v.x; ids[4 * q + 1] = v.y; ids[4 * q + 2] = v.z; ids[4 * q + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < KM; ++j) ids[j] = (tp < n && j < k) ? __ldg(src + j) : -1;
+        }
+    }
+    for (int e = tid; e < E; e += kThreads) {
+        s_before[e] = 0;
+        s_total[e] = 0;
+    }
+    if (tid < 32) s_mask[tid] = 0;
+    if (tid < 33) s_cnt[tid] = 0;
+    __syncthreads();
+    uint32_t hits = 0;
+    int valid = 0;
+    if (tp < n) {
+        int32_t *cnt = tp < t ? s_before : s_total;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            const int32_t e = ids[j];
+            if (j < k && (uint32_t)e < (uint32_t)E) {
+                red_shared_add(cnt + e, 1);
+                ++valid;
+                const int r = div_small(e, rm);
+                const int d = r - b;
+                if (d >= 0) {
+                    const int q = div_small(d, gm);
+                    if (q * G == d && q < nd) hits |= 1u << q;
+                }
+                if (tp == t) atomicOr(&s_mask[r >> 5], 1u << (r & 31));
+            }
+        }
+        if (tp == t) {
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (j < k) s_own[j] = ids[j];
+        }
+    }
+    valid = __reduce_add_sync(0xFFFFFFFFu, valid);
+    if (lane == 0 && valid) red_shared_add(&s_cnt[0], valid);
+    for (int i = 0; i < nd; ++i) {   // block-uniform
+        const int c = __popc(__ballot_sync(0xFFFFFFFFu, (hits >> i) & 1u));
+        if (lane == 0 && c) red_shared_add(&s_cnt[1 + i], c);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kThreads) s_total[e] += s_before[e];
+    if (G > 1) {
+        if (tid < nd) tokens_per_rank[b + tid * G] = s_cnt[1 + tid];
+    } else {
+        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = (int32_t)((s_mask[r >> 5] >> (r & 31)) & 1u);
+    }
+    if (has_tok)
+        for (int r = tid; r < R; r += kThreads)
+            in_rank[t * R + r] = (uint8_t)((s_mask[r >> 5] >> (r & 31)) & 1u);
+    __syncthreads();
+    const int32_t m_total = s_cnt[0];
+
+    // own rows: slot j ranked by warp j % 8 (an empty batch's single CTA has none)
+    bool over = false, bad = false;
+    for (int j = warp; has_tok && j < k; j += kWarps) {   // warp-uniform
+        const int32_t e = s_own[j];
+        int32_t row = -1;
+        if ((uint32_t)e < (uint32_t)E) {
+            int32_t below = 0;
+            if (cap == 0)
+                for (int q = lane; q < e; q += 32) below += s_total[q];
+            below = __reduce_add_sync(0xFFFFFFFFu, below);
+            int dup = 0;
+            for (int jj = 0; jj < j; ++jj) dup += s_own[jj] == e ? 1 : 0;
+            const int32_t rank = s_before[e] + dup;
+            if (cap > 0) {
+                if (rank >= cap) over = true;
+                else row = e * cap + rank;
+            } else {
+                row = below + rank;
+            }
+            if (row >= recv_rows) { bad = true; row = -1; }
+        } else if (e != -1) {
+            bad = true;
+        }
+        if (lane == 0) {
+            s_row[j] = row;
+            dst_pos[t * k + j] = row;
+            if (row >= 0) recv_src[row] = (int32_t)(t * k + j);
+        }
+    }
+    if (lane == 0 && over) report(status, kErrCapacity);
+    if (lane == 0 && bad) report(status, kErrRange);
+
+    // CTA 0: counts, offsets, max
+    if (b == 0) {
+        const int32_t tot = block_exclusive_scan(s_total, s_off, E, scan_tmp);
+        int32_t mx = 0;
+        for (int e = tid; e < E; e += kThreads) {
+            tokens_per_expert[e] = s_total[e];
+            expert_offset[e] = s_off[e];
+            mx = max(mx, s_total[e]);
+        }
+        if (tid == 0) expert_offset[E] = tot;
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) scan_tmp[warp] = mx;
+        __syncthreads();
+        if (tid == 0) {
+            int32_t m = 0;
+            for (int w = 0; w < kWarps; ++w) m = max(m, scan_tmp[w]);
+            *max_count = m;
+        }
+    }
+    // this CTA's share of the rows that receive nothing
+    const int64_t fstep = (int64_t)G * kThreads;
+    if (cap > 0) {
+        for (int64_t i = (int64_t)b * kThreads + tid; i < (int64_t)E * cap; i += fstep) {
+            const int e = (int)(i / cap);
+            if (i - (int64_t)e * cap >= s_total[e]) recv_src[i] = -1;
+        }
+    } else {
+        for (int64_t i = m_total + (int64_t)b * kThreads + tid; i < n * k; i += fstep) recv_src[i] = -1;
+    }
+    __syncthreads();   // s_row
+
+    // the token's FP8 rows: 16 values per thread per pass, 8 lanes per scale block
+    if (!has_tok) return;
+    const int chunks = h >> 4, nblk = h >> 7;
+    for (int c0 = warp * 32; c0 < chunks; c0 += kThreads) {   // warp-uniform
+        const int c = c0 + lane;
+        const bool active = c < chunks;
+        uint4 a = make_uint4(0, 0, 0, 0), bb = a;
+        if (active) {
+            a = ld_nc_v4(x + t * h + (int64_t)c * 16);
+            bb = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
+        }
+        float m = absmax16(a, bb);
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        if (!active) continue;
+        const float amax_c = fmaxf(m, 1e-4f);
+        float scale, inv;
+        block_scale(amax_c, pow2 != 0, scale, inv);
+        const uint4 q = quant16(a, bb, inv);
+        for (int j = 0; j < k; ++j) {
+            const int32_t row = s_row[j];
+            if (row < 0) continue;
+            st_cs_v4(recv_x + (int64_t)row * h + (int64_t)c * 16, q);
+            if ((c & 7) == 0) recv_scale[(int64_t)row * nblk + (c >> 3)] = scale;
+        }
+    }
+}
+
 // ------------------------------------------- fused layout + FP8 dispatch
 //
 // Prefill-sized batches: the layout and the FP8 dispatch in one launch, one
@@ -1882,9 +2078,20 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
     const int sms = device_sm_count();
     if (sms <= 0) return CGL_ECUDA;
     const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+    const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+    if (n <= use_sms && n <= kThreads && (n <= 1 || rep_designated(0, (int)n, R) <= 32)) {
+        const dim3 grid((unsigned)(n < 1 ? 1 : n));
+        const cudaError_t e2 =
+            k <= 8 ? launch_pdl(decode_token_kernel<8>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap, vec, x,
+                                h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
+                                recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status)
+                   : launch_pdl(decode_token_kernel<kMaxTopk>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap,
+                                vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
+                                dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
+        return e2 == cudaSuccess ? CGL_OK : CGL_ECUDA;
+    }
     const DecodeShape d = decode_shape(n, k, R, use_sms);
     const size_t smem = (rep_smem_words(d.T, E, R) + (size_t)d.T * k) * sizeof(int32_t);
-    const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
     cudaError_t err;
     switch (d.CH) {
         case 1:

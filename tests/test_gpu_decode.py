@@ -84,3 +84,23 @@ def test_fused_decode_in_a_graph(oracle_mod):
         used = L.recv_src >= 0
         assert np.array_equal(rx.cpu().numpy()[used], ox[used])
     del g
+
+
+@pytest.mark.parametrize("n,k,E,R", [(0, 8, 256, 32), (1, 8, 256, 32), (2, 8, 256, 64), (5, 8, 256, 256),
+                                     (64, 8, 512, 512), (148, 3, 48, 12), (30, 32, 64, 8)])
+def test_fused_decode_one_token_per_cta_shapes(oracle_mod, n, k, E, R):
+    """Batches of at most one token per SM take one CTA per token: empty and
+    one-token batches, more ranks than one CTA's 32 designated ranks (the
+    general kernel then), k that is not a multiple of 4, top-32, and repeated
+    experts inside tokens; compact, padded and overflowing."""
+    rng = np.random.default_rng(n * 13 + k + E)
+    h = 256
+    x = W.f32_to_bf16_bits(rng.standard_normal((n, h)).astype(np.float32))
+    idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    if n:
+        idx[rng.random((n, k)) < 0.05] = -1
+    _check(oracle_mod, x, idx, E, R, 0)
+    mc = int(oracle_mod.get_layout(idx, E, R).max_count) if n else 0
+    _check(oracle_mod, x, idx, E, R, max(1, mc))
+    if mc > 1:
+        _check(oracle_mod, x, idx, E, R, mc - 1)
