@@ -1228,9 +1228,10 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 // scan outside CTA 0), rank = before[e] + the earlier slots of the token with
 // that expert.  CTA 0 writes the expert counts, offsets and max; every CTA
 // writes its token's rows, is_token_in_rank row and share of the recv_src
-// fill, then quantises the token as the fused decode kernel does.  About five
-// block barriers where the general block takes a dozen.
-template <int KM>
+// fill, then (kDispatch) quantises the token as the fused decode kernel does.
+// About five block barriers where the general block takes a dozen.  The
+// layout-only instance serves cgl_get_layout for such batches.
+template <int KM, bool kDispatch>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int vec,
                     const uint16_t *__restrict__ x, int h, int32_t *__restrict__ tokens_per_expert,
@@ -1385,7 +1386,7 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     __syncthreads();   // s_row
 
     // the token's FP8 rows: 16 values per thread per pass, 8 lanes per scale block
-    if (!has_tok) return;
+    if (!kDispatch || !has_tok) return;
     const int chunks = h >> 4, nblk = h >> 7;
     for (int c0 = warp * 32; c0 < chunks; c0 += kThreads) {   // warp-uniform
         const int c = c0 + lane;
@@ -1864,6 +1865,31 @@ cgl_status ld_launch(const LdShape &sh, const int32_t *idx, int64_t n, int k, in
 
 }  // namespace
 
+// One CTA per token: at most one token per SM in use (and per thread of the
+// scanning block), at most 32 designated ranks per CTA, E within the static
+// shared histograms.
+bool token_layout_fits(int64_t n, int k, int E, int R, int use_sms) {
+    (void)k;
+    return n <= use_sms && n <= kThreads && E <= kMaxExperts && (n <= 1 || rep_designated(0, (int)n, R) <= 32);
+}
+
+template <bool kDispatch>
+cgl_status launch_token_kernel(const int32_t *idx, int64_t n, int k, int E, int R, int cap, int vec,
+                               const uint16_t *x, int h, int32_t *tokens_per_expert, int32_t *tokens_per_rank,
+                               uint8_t *in_rank, int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
+                               int32_t *recv_src, int64_t recv_rows, uint8_t *recv_x, float *recv_scale, bool pow2,
+                               uint32_t *status, cudaStream_t stream) {
+    const dim3 grid((unsigned)(n < 1 ? 1 : n));
+    const cudaError_t err =
+        k <= 8 ? launch_pdl(decode_token_kernel<8, kDispatch>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap,
+                            vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
+                            recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status)
+               : launch_pdl(decode_token_kernel<kMaxTopk, kDispatch>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R,
+                            cap, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
+                            dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
+    return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
+}
+
 size_t layout_workspace_bytes(int64_t n, int k, int E, int R) { return ws_layout(n, k, E, R).bytes; }
 
 size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
@@ -1871,6 +1897,9 @@ size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
 }
 
 bool layout_dispatch_fused_fits(int64_t n, int k, int E, int R, int h, int num_sms) {
+    const int sms = device_sm_count();
+    const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+    if (sms > 0 && token_layout_fits(n, k, E, R, use_sms)) return true;
     return ld_fits(ld_shape(n, k, E, R, h, num_sms));
 }
 
@@ -1880,6 +1909,18 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                       int32_t *max_count, int32_t *dst_pos, int32_t *recv_src, uint8_t *recv_x,
                                       float *recv_scale, void *ws, int num_sms, bool pow2, uint32_t *status,
                                       cudaStream_t stream) {
+    {   // at most one token per SM: one CTA per token does both
+        const int sms = device_sm_count();
+        if (sms <= 0) return CGL_ECUDA;
+        const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
+        if (token_layout_fits(n, k, E, R, use_sms)) {
+            const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
+            const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+            return launch_token_kernel<true>(idx, n, k, E, R, cap, vec, x, h, tokens_per_expert, tokens_per_rank,
+                                             in_rank, expert_offset, max_count, dst_pos, recv_src, recv_rows, recv_x,
+                                             recv_scale, pow2, status, stream);
+        }
+    }
     const LdShape sh = ld_shape(n, k, E, R, h, num_sms);
     if (ld_fits(sh)) {
         switch (sh.CH) {
@@ -1908,7 +1949,10 @@ bool layout_needs_smem_optin(int E, int R, int k) {
     return smem_words(0, k, E, R) * sizeof(int32_t) > kSmemDefault;
 }
 
-bool layout_fused_fits(int64_t n, int k, int E, int R) { return rep_grid(n, k, E, R) > 0 || fused_fits<false>(n, k, E, R); }
+bool layout_fused_fits(int64_t n, int k, int E, int R) {
+    const int sms = device_sm_count();
+    return (sms > 0 && token_layout_fits(n, k, E, R, sms)) || rep_grid(n, k, E, R) > 0 || fused_fits<false>(n, k, E, R);
+}
 
 template <bool kRankKeys, int CH>
 cgl_status launch_layout_ch(const int32_t *idx, int64_t n, int k, int E_ids, int R, int cap,
@@ -1968,6 +2012,14 @@ cgl_status launch_layout_impl(const int32_t *idx, int64_t n, int k, int E_ids, i
                               int32_t *recv_src, void *ws, uint32_t *status, cudaStream_t stream) {
     const int nkeys = kRankKeys ? R : E_ids;
     if constexpr (!kRankKeys) {
+        const int sms = device_sm_count();
+        if (sms > 0 && token_layout_fits(n, k, E_ids, R, sms)) {
+            const int64_t recv_rows = cap > 0 ? (int64_t)E_ids * cap : n * k;
+            const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
+            return launch_token_kernel<false>(idx, n, k, E_ids, R, cap, vec, nullptr, 0, tokens_per_key,
+                                              tokens_per_rank, in_rank, key_offset, max_count, dst_pos, recv_src,
+                                              recv_rows, nullptr, nullptr, false, status, stream);
+        }
         const int G = rep_grid(n, k, E_ids, R);
         if (G > 0) {
             const int T = tokens_per_block(k, 1);
@@ -2079,17 +2131,10 @@ cgl_status launch_decode_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
     if (sms <= 0) return CGL_ECUDA;
     const int use_sms = (num_sms > 0 && num_sms < sms) ? num_sms : sms;
     const int vec = (k % 4 == 0) && (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
-    if (n <= use_sms && n <= kThreads && (n <= 1 || rep_designated(0, (int)n, R) <= 32)) {
-        const dim3 grid((unsigned)(n < 1 ? 1 : n));
-        const cudaError_t e2 =
-            k <= 8 ? launch_pdl(decode_token_kernel<8>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap, vec, x,
-                                h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
-                                recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status)
-                   : launch_pdl(decode_token_kernel<kMaxTopk>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap,
-                                vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
-                                dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
-        return e2 == cudaSuccess ? CGL_OK : CGL_ECUDA;
-    }
+    if (token_layout_fits(n, k, E, R, use_sms))
+        return launch_token_kernel<true>(idx, n, k, E, R, cap, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank,
+                                         expert_offset, max_count, dst_pos, recv_src, recv_rows, recv_x, recv_scale,
+                                         pow2, status, stream);
     const DecodeShape d = decode_shape(n, k, R, use_sms);
     const size_t smem = (rep_smem_words(d.T, E, R) + (size_t)d.T * k) * sizeof(int32_t);
     cudaError_t err;

@@ -200,10 +200,11 @@ def test_layout_replicated_counts_with_unaligned_ids(oracle_mod):
     assert st.item() == 0
 
 
-@pytest.mark.parametrize("n,k,E,R", [(64, 8, 256, 128), (250, 4, 512, 256)])
+@pytest.mark.parametrize("n,k,E,R", [(200, 8, 256, 256), (250, 4, 512, 256)])
 def test_layout_cluster_path_many_ranks(oracle_mod, n, k, E, R):
-    """More ranks than 32 per block of the replicated-count layout: these small
-    batches take the thread-block-cluster layout instead."""
+    """More tokens than SMs, and more ranks than 32 per block of the
+    replicated-count layout: these small batches take the thread-block-cluster
+    layout instead."""
     rng = np.random.default_rng(n + R)
     idx = rng.integers(0, E, (n, k)).astype(np.int32)
     idx[rng.random((n, k)) < 0.05] = -1

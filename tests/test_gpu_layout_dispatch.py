@@ -60,8 +60,10 @@ def test_layout_dispatch_fp8_takes_one_launch_at_prefill():
     assert cgl.layout_dispatch_kernel_count(wl.num_tokens, wl.topk, wl.num_experts, wl.num_ranks, wl.hidden) == 1
     # 16384 tokens at hidden 7168: 111 per CTA do not fit in shared memory -> separate kernels
     assert cgl.layout_dispatch_kernel_count(16384, 8, 256, 64, 7168) > 1
-    # 128 tokens: too few pairs per SM -> separate kernels
-    assert cgl.layout_dispatch_kernel_count(128, 8, 256, 32, 7168) > 1
+    # 128 tokens, at most one per SM: one CTA per token does layout and dispatch
+    assert cgl.layout_dispatch_kernel_count(128, 8, 256, 32, 7168) == 1
+    # 1000 tokens: too few pairs per SM for the fused prefill kernel -> layout, then dispatch
+    assert cgl.layout_dispatch_kernel_count(1000, 8, 256, 64, 7168) > 1
 
 
 def test_layout_dispatch_fp8_fused_on_fewer_sms(oracle_mod):
