@@ -1230,9 +1230,11 @@ decode_fused_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 // writes its token's rows, is_token_in_rank row and share of the recv_src
 // fill, then (kDispatch) quantises the token as the fused decode kernel does.
 // About five block barriers where the general block takes a dozen.  The
-// layout-only instance serves cgl_get_layout for such batches.
-template <int KM, bool kDispatch>
-__global__ void __launch_bounds__(kThreads, 1)
+// dispatching instance runs 512 threads, so one pass quantises a 7168-value
+// token (the layout phases use threads 0-255); the layout-only instance (256
+// threads) serves cgl_get_layout for such batches.
+template <int KM, bool kDispatch, int NT>
+__global__ void __launch_bounds__(NT, 1)
 decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, int vec,
                     const uint16_t *__restrict__ x, int h, int32_t *__restrict__ tokens_per_expert,
                     int32_t *__restrict__ tokens_per_rank, uint8_t *__restrict__ in_rank,
@@ -1271,7 +1273,7 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
             for (int j = 0; j < KM; ++j) ids[j] = (tp < n && j < k) ? __ldg(src + j) : -1;
         }
     }
-    for (int e = tid; e < E; e += kThreads) {
+    for (int e = tid; e < E; e += NT) {
         s_before[e] = 0;
         s_total[e] = 0;
     }
@@ -1310,21 +1312,21 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         if (lane == 0 && c) red_shared_add(&s_cnt[1 + i], c);
     }
     __syncthreads();
-    for (int e = tid; e < E; e += kThreads) s_total[e] += s_before[e];
+    for (int e = tid; e < E; e += NT) s_total[e] += s_before[e];
     if (G > 1) {
         if (tid < nd) tokens_per_rank[b + tid * G] = s_cnt[1 + tid];
     } else {
-        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = (int32_t)((s_mask[r >> 5] >> (r & 31)) & 1u);
+        for (int r = tid; r < R; r += NT) tokens_per_rank[r] = (int32_t)((s_mask[r >> 5] >> (r & 31)) & 1u);
     }
     if (has_tok)
-        for (int r = tid; r < R; r += kThreads)
+        for (int r = tid; r < R; r += NT)
             in_rank[t * R + r] = (uint8_t)((s_mask[r >> 5] >> (r & 31)) & 1u);
     __syncthreads();
     const int32_t m_total = s_cnt[0];
 
     // own rows: slot j ranked by warp j % 8 (an empty batch's single CTA has none)
     bool over = false, bad = false;
-    for (int j = warp; has_tok && j < k; j += kWarps) {   // warp-uniform
+    for (int j = warp; has_tok && j < k; j += NT / 32) {   // warp-uniform
         const int32_t e = s_own[j];
         int32_t row = -1;
         if ((uint32_t)e < (uint32_t)E) {
@@ -1354,18 +1356,20 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     if (lane == 0 && over) report(status, kErrCapacity);
     if (lane == 0 && bad) report(status, kErrRange);
 
-    // CTA 0: counts, offsets, max
+    // CTA 0: counts, offsets, max (threads 0-255: the scan's barrier is hardware barrier 1)
     if (b == 0) {
-        const int32_t tot = block_exclusive_scan(s_total, s_off, E, scan_tmp);
-        int32_t mx = 0;
-        for (int e = tid; e < E; e += kThreads) {
-            tokens_per_expert[e] = s_total[e];
-            expert_offset[e] = s_off[e];
-            mx = max(mx, s_total[e]);
+        if (tid < kThreads) {
+            const int32_t tot = block_exclusive_scan(s_total, s_off, E, scan_tmp);
+            int32_t mx = 0;
+            for (int e = tid; e < E; e += kThreads) {
+                tokens_per_expert[e] = s_total[e];
+                expert_offset[e] = s_off[e];
+                mx = max(mx, s_total[e]);
+            }
+            if (tid == 0) expert_offset[E] = tot;
+            mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+            if (lane == 0) scan_tmp[warp] = mx;
         }
-        if (tid == 0) expert_offset[E] = tot;
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (lane == 0) scan_tmp[warp] = mx;
         __syncthreads();
         if (tid == 0) {
             int32_t m = 0;
@@ -1374,21 +1378,21 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
         }
     }
     // this CTA's share of the rows that receive nothing
-    const int64_t fstep = (int64_t)G * kThreads;
+    const int64_t fstep = (int64_t)G * NT;
     if (cap > 0) {
-        for (int64_t i = (int64_t)b * kThreads + tid; i < (int64_t)E * cap; i += fstep) {
+        for (int64_t i = (int64_t)b * NT + tid; i < (int64_t)E * cap; i += fstep) {
             const int e = (int)(i / cap);
             if (i - (int64_t)e * cap >= s_total[e]) recv_src[i] = -1;
         }
     } else {
-        for (int64_t i = m_total + (int64_t)b * kThreads + tid; i < n * k; i += fstep) recv_src[i] = -1;
+        for (int64_t i = m_total + (int64_t)b * NT + tid; i < n * k; i += fstep) recv_src[i] = -1;
     }
     __syncthreads();   // s_row
 
     // the token's FP8 rows: 16 values per thread per pass, 8 lanes per scale block
     if (!kDispatch || !has_tok) return;
     const int chunks = h >> 4, nblk = h >> 7;
-    for (int c0 = warp * 32; c0 < chunks; c0 += kThreads) {   // warp-uniform
+    for (int c0 = warp * 32; c0 < chunks; c0 += NT) {   // warp-uniform
         const int c = c0 + lane;
         const bool active = c < chunks;
         uint4 a = make_uint4(0, 0, 0, 0), bb = a;
@@ -1879,12 +1883,13 @@ cgl_status launch_token_kernel(const int32_t *idx, int64_t n, int k, int E, int 
                                uint8_t *in_rank, int32_t *expert_offset, int32_t *max_count, int32_t *dst_pos,
                                int32_t *recv_src, int64_t recv_rows, uint8_t *recv_x, float *recv_scale, bool pow2,
                                uint32_t *status, cudaStream_t stream) {
+    constexpr int NT = kDispatch ? 2 * kThreads : kThreads;
     const dim3 grid((unsigned)(n < 1 ? 1 : n));
     const cudaError_t err =
-        k <= 8 ? launch_pdl(decode_token_kernel<8, kDispatch>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R, cap,
+        k <= 8 ? launch_pdl(decode_token_kernel<8, kDispatch, NT>, grid, dim3(NT), 0, stream, idx, n, k, E, R, cap,
                             vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count, dst_pos,
                             recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status)
-               : launch_pdl(decode_token_kernel<kMaxTopk, kDispatch>, grid, dim3(kThreads), 0, stream, idx, n, k, E, R,
+               : launch_pdl(decode_token_kernel<kMaxTopk, kDispatch, NT>, grid, dim3(NT), 0, stream, idx, n, k, E, R,
                             cap, vec, x, h, tokens_per_expert, tokens_per_rank, in_rank, expert_offset, max_count,
                             dst_pos, recv_src, recv_rows, recv_x, recv_scale, (int)pow2, status);
     return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
