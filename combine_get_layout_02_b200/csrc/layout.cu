@@ -222,27 +222,39 @@ template <int CH = kChunks>
 __device__ __forceinline__ int pair_of(int i) { return (threadIdx.x >> 5) * (CH * 32) + i * 32 + (threadIdx.x & 31); }
 
 // Load this thread's ids (coalesced: each warp reads 32 consecutive ids per
-// chunk) of block `token_block` (T tokens per block).  Returns true if an id
-// outside [-1, E_ids) was seen (such slots make no copy).
+// chunk) of block `token_block` (T tokens per block).  Nothing waits for the
+// loads here: check_pairs is the first use.
 template <int CH = kChunks>
-__device__ __forceinline__ bool load_pairs(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids,
-                                           int64_t token_block, int T, PairsT<CH> &P) {
+__device__ __forceinline__ void load_pairs_only(const int32_t *__restrict__ idx, int64_t n, int k,
+                                                int64_t token_block, int T, PairsT<CH> &P) {
     P.t0 = token_block * T;
     const int64_t rem = n - P.t0;
     P.nt = rem <= 0 ? 0 : (rem < T ? (int)rem : T);
     P.np = P.nt * k;
     const int32_t *src = idx + P.t0 * k;
-    bool bad = false;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
         const int p = pair_of<CH>(i);
         P.e[i] = p < P.np ? __ldg(src + p) : -1;
     }
+}
+
+// Returns true if an id outside [-1, E_ids) was loaded; such slots make no copy.
+template <int CH = kChunks>
+__device__ __forceinline__ bool check_pairs(int E_ids, PairsT<CH> &P) {
+    bool bad = false;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
         if (P.e[i] < -1 || P.e[i] >= E_ids) { bad = true; P.e[i] = -1; }
     }
     return bad;
+}
+
+template <int CH = kChunks>
+__device__ __forceinline__ bool load_pairs(const int32_t *__restrict__ idx, int64_t n, int k, int E_ids,
+                                           int64_t token_block, int T, PairsT<CH> &P) {
+    load_pairs_only<CH>(idx, n, k, token_block, T, P);
+    return check_pairs<CH>(E_ids, P);
 }
 
 // Turn the loaded ids into keys and rank the keys within the warp.  Expert
@@ -989,6 +1001,17 @@ __host__ __device__ __forceinline__ int rep_designated(int b, int G, int R) {
     return b < R ? (R - 1 - b) / G + 1 : 0;
 }
 
+// Ask the TMA engine to bring the ids of the block's tokens [t0, t0 + T) into
+// L2 (one thread).  Every block reads every id in its scan; with each block
+// fetching its own share first, those reads hit L2 instead of queueing in HBM
+// behind the block's other traffic.  kVec-aligned ids only (16-byte aligned,
+// k % 4 == 0), so the range is 16-byte aligned and sized.
+__device__ __forceinline__ void prefetch_own_ids(const int32_t *idx, int64_t n, int k, int64_t t0, int T,
+                                                 bool vec) {
+    const int64_t nt = t0 < n ? (n - t0 < T ? n - t0 : T) : 0;
+    if (vec && threadIdx.x == 0 && nt > 0) prefetch_l2_bulk(idx + t0 * k, (uint32_t)(nt * k * 4));
+}
+
 // Every id of the batch into before[] (tokens < t0) / rest[] (tokens >= t0),
 // and distinct tokens of the designated ranks b + i G (i < nd <= 32) into
 // dcnt[i].  Warp-uniform loop over groups of 32 tokens, one token per lane;
@@ -1077,13 +1100,17 @@ __device__ void rep_zero(int T, int E, int R, const Smem &s) {
 }
 
 // The block's own part of a replicated-count layout once the scan's counts are
-// in shared memory, run by the 256 threads of warps 0-7 (barrier 1): block b =
-// blockIdx.x of G = gridDim.x owns tokens [b T, b T + T).  Ranks its own copies,
-// writes every layout output of its own tokens, its designated ranks'
-// tokens_per_rank, its share of the recv_src fill, and (block 0) the expert
-// counts, offsets and max; s_dst (optional, shared, T k words) also receives its
-// rows.  P holds the block's ids (load_pairs).  Requires G == 1 or
-// rep_designated(0, G, R) <= 32.
+// in shared memory (s.base: copies before the block, s.total: the rest, s.part:
+// designated-rank counts), run by the 256 threads of warps 0-7 (barrier 1):
+// block b = blockIdx.x of G = gridDim.x owns tokens [b T, b T + T).  Ranks its
+// own copies, writes every layout output of its own tokens, its designated
+// ranks' tokens_per_rank, its share of the recv_src fill, and (block 0) the
+// expert counts, offsets and max; s_dst (optional, shared, T k words) also
+// receives its rows.  P holds the block's ids (load_pairs_only, then checked
+// here).  Three barriers: after the warp ranks and rank sets; after the warp
+// offsets, the warps' scans of the expert totals and the is_token_in_rank
+// rows; after the bases.  scan_tmp: 2 kWarps words.
+// Requires G == 1 or rep_designated(0, G, R) <= 32.
 template <int CH>
 __device__ void rep_finish(const int32_t *__restrict__ idx, int64_t n, int k, int E, int R, int cap, bool bad,
                            PairsT<CH> &P, int32_t *__restrict__ tokens_per_expert,
@@ -1091,26 +1118,93 @@ __device__ void rep_finish(const int32_t *__restrict__ idx, int64_t n, int k, in
                            int32_t *__restrict__ expert_offset, int32_t *__restrict__ max_count,
                            int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
                            uint32_t *status, const Smem &s, int32_t *scan_tmp, int32_t *s_dst) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, b = blockIdx.x;
     const int nd = G > 1 ? rep_designated(b, G, R) : 0;
     key_and_rank<false, CH>(idx, k, E, E / R, E, s, P);
     rank_sets<CH>(k, E, R, s, P);
-    lsync();
-    warp_offsets(E, s);
-    if (G == 1) rank_counts<CH>(k, R, s, P);   // one block: its own tokens are all tokens
-    for (int e = tid; e < E; e += kThreads) s.total[e] += s.base[e];   // rest + before
-    lsync();
-    write_rank_rows<CH>(R, in_rank, s, P);
-    if (G == 1) {
-        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
-    } else if (tid < nd) {
-        tokens_per_rank[b + tid * G] = s.part[tid];
-    }
     if (lsync_or(bad) && tid == 0) report(status, kErrRange);
-    bases_and_rows<true, false, CH, true>(nullptr, nullptr, n, k, E, R, cap, recv_rows, tokens_per_expert, nullptr,
-                                          expert_offset, max_count, dst_pos, recv_src, status, s, P, scan_tmp,
-                                          s_dst);
+    warp_offsets(E, s);
+    // expert totals (rest + before) and their exclusive scan: thread tid takes
+    // experts [i0, i1), a warp scans its threads' sums, scan_tmp[w] holds warp
+    // w's total and scan_tmp[kWarps + w] its largest count
+    const int per = (E + kThreads - 1) / kThreads;
+    const int i0 = min(E, tid * per), i1 = min(E, i0 + per);
+    int32_t local = 0, mx = 0;
+    for (int i = i0; i < i1; ++i) {
+        const int32_t t = s.total[i] + s.base[i];
+        s.total[i] = t;
+        local += t;
+        mx = max(mx, t);
+    }
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 31) scan_tmp[warp] = incl;
+    if (lane == 0) scan_tmp[kWarps + warp] = mx;
+    if (G == 1) rank_counts<CH>(k, R, s, P);   // one block: its own tokens are all tokens
+    else if (tid < nd) tokens_per_rank[b + tid * G] = s.part[tid];
+    write_rank_rows<CH>(R, in_rank, s, P);
+    lsync();
+    int32_t run = incl - local, m_total = 0, m_max = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const int32_t v = scan_tmp[w];
+        if (w < warp) run += v;
+        m_total += v;
+        m_max = max(m_max, scan_tmp[kWarps + w]);
+    }
+    for (int i = i0; i < i1; ++i) {
+        const int32_t t = s.total[i];
+        s.base[i] += cap > 0 ? i * cap : run;
+        if (b == 0) {
+            tokens_per_expert[i] = t;
+            expert_offset[i] = run;
+        }
+        run += t;
+    }
+    if (b == 0 && tid == 0) {
+        expert_offset[E] = m_total;
+        *max_count = m_max;
+    }
+    if (G == 1)
+        for (int r = tid; r < R; r += kThreads) tokens_per_rank[r] = s.hr[r];
+    lsync();
+    const int64_t step = (int64_t)G * kThreads;
+    if (cap > 0) {   // rows past an expert's copies
+        const int64_t rows = (int64_t)E * cap;
+        for (int64_t i = (int64_t)b * kThreads + tid; i < rows; i += step) {
+            const int e = (int)(i / cap);
+            if (i - (int64_t)e * cap >= s.total[e]) recv_src[i] = -1;
+        }
+    } else {         // rows past the last copy (ids of -1)
+        for (int64_t i = m_total + (int64_t)b * kThreads + tid; i < n * k; i += step) recv_src[i] = -1;
+    }
+    bool over = false, bad_row = false;
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int p = pair_of<CH>(i);
+        if (p >= P.np) continue;
+        const int32_t e = P.e[i];
+        int32_t d = -1;
+        if (e >= 0) {
+            const int32_t pos = s.base[e] + s.wc[warp * E + e] + P.rk[i];
+            if (cap > 0 && pos - e * cap >= cap) over = true;
+            else if (pos >= recv_rows) bad_row = true;
+            else d = pos;
+        }
+        const int64_t q = P.t0 * k + p;
+        dst_pos[q] = d;
+        if (s_dst) s_dst[p] = d;
+        if (d >= 0) recv_src[d] = (int32_t)q;   // the row's source slot t k + j
+    }
+    if (over) report(status, kErrCapacity);
+    if (bad_row) report(status, kErrRange);
 }
 
 // A whole replicated-count layout block run by the 256 threads of warps 0-7.
@@ -1122,10 +1216,11 @@ __device__ void rep_layout_block(const int32_t *__restrict__ idx, int64_t n, int
                                  int32_t *__restrict__ dst_pos, int32_t *__restrict__ recv_src, int64_t recv_rows,
                                  uint32_t *status, const Smem &s, int32_t *scan_tmp, int32_t *s_dst) {
     PairsT<CH> P;
-    const bool bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight while zeroing
+    load_pairs_only<CH>(idx, n, k, blockIdx.x, T, P);   // in flight while zeroing and scanning
     rep_zero<kThreads>(T, E, R, s);
     lsync();
     rep_scan<kThreads>(idx, n, k, E, R, P.t0, vec, s);
+    const bool bad = check_pairs<CH>(E, P);
     rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
                    max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
 }
@@ -1149,14 +1244,13 @@ layout_rep_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int 
     const Smem s = carve_rep(smem_rep, T, E, R);
     griddep_wait();   // the ids, and readers of the outputs, may be the kernels just before
     PairsT<CH> P;
-    bool bad = false;
-    if (threadIdx.x < kThreads) bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight
+    if (threadIdx.x < kThreads) load_pairs_only<CH>(idx, n, k, blockIdx.x, T, P);   // in flight
     rep_zero<NT>(T, E, R, s);
     __syncthreads();
     rep_scan<NT>(idx, n, k, E, R, (int64_t)blockIdx.x * T, vec != 0, s);
     __syncthreads();
     if (threadIdx.x < kThreads)
-        rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
                        max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, nullptr);
 }
 
@@ -1623,6 +1717,7 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
     const int ng = cnt0 < kMaxGroups ? (cnt0 > 0 ? cnt0 : 1) : kMaxGroups;
     const int split = cnt0 - (cnt0 * kLateShareNum) / kLateShareDen;   // warps 1-7 stage [split, cnt0)
     griddep_wait();   // ids and x may come from the kernels just before, which may still read our outputs
+    prefetch_own_ids(idx, n, k, t0, T, vec != 0);   // ahead of x in the memory queues
     if (threadIdx.x < 32 && cnt0 > 0) {
         // the CTA's x rows are one contiguous range: the TMA engine streams it from
         // HBM into L2 while the ids are scanned, so the staging loads hit L2
@@ -1632,14 +1727,13 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
             prefetch_l2_bulk(src + off, (uint32_t)(bytes - off < kPrefetchBytes ? bytes - off : kPrefetchBytes));
     }
     PairsT<CH> P;
-    bool bad = false;
-    if (threadIdx.x < kThreads) bad = load_pairs<CH>(idx, n, k, E, blockIdx.x, T, P);   // in flight
+    if (threadIdx.x < kThreads) load_pairs_only<CH>(idx, n, k, blockIdx.x, T, P);   // in flight
     rep_zero<kLdThreads>(T, E, R, s);
     __syncthreads();
     rep_scan<kLdThreads>(idx, n, k, E, R, t0, vec != 0, s);
     __syncthreads();
     if (threadIdx.x < kThreads) {
-        rep_finish<CH>(idx, n, k, E, R, cap, bad, P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
+        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
                        max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
         lsync();   // every row of the block is in s_dst
         if (threadIdx.x < 32) {
