@@ -210,3 +210,23 @@ def test_layout_cluster_path_many_ranks(oracle_mod, n, k, E, R):
     idx[rng.random((n, k)) < 0.05] = -1
     lay, _ = run_both(oracle_mod, idx, E, R, 0)
     run_both(oracle_mod, idx, E, R, max(1, int(lay.max_count.item()) - 1))
+
+
+@pytest.mark.parametrize("n,k,E,R,cap", [(4000, 8, 256, 64, 0), (4096, 8, 1024, 1024, 0), (1000, 32, 256, 64, 0),
+                                         (3001, 6, 96, 8, 0), (4096, 8, 256, 64, -1), (2049, 4, 64, 64, 0)])
+def test_layout_replicated_counts_wide_blocks(oracle_mod, n, k, E, R, cap):
+    """Batches of 4097 to 32768 (token, slot) pairs take the replicated-count
+    layout with 1024-thread blocks: ragged last blocks, many designated ranks
+    per block, top-32, a top-k that is not a multiple of 4 (scalar id loads)
+    and padded receive rows, at and below the largest per-expert count."""
+    rng = np.random.default_rng(n * 7 + k)
+    if k <= E:
+        idx = np.argsort(rng.random((n, E)), axis=1)[:, :k].astype(np.int32)
+    else:
+        idx = rng.integers(0, E, (n, k)).astype(np.int32)
+    idx[rng.random((n, k)) < 0.03] = -1
+    assert 4096 < n * k <= 32768
+    lay, ref = run_both(oracle_mod, idx, E, R, 0)
+    if cap < 0:
+        run_both(oracle_mod, idx, E, R, int(lay.max_count.item()))
+        run_both(oracle_mod, idx, E, R, max(1, int(lay.max_count.item()) - 2))
