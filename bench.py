@@ -43,10 +43,10 @@ FALLBACK_HBM_GBS = 6650.0
 # source and the shared device header it was taken on; a changed source
 # reports traffic null.
 NCU_TRAFFIC = {
-    "combine": {"bytes": 507093760, "src_sha": "e63c09f116de7be3"},
-    "dispatch_fp8": {"bytes": 243200256, "src_sha": "6c478e0bec1a7510"},
-    "layout+dispatch_fp8": {"bytes": 250198016, "src_sha": "909cacef0c241f29"},
-    "layout": {"bytes": 217600, "src_sha": "909cacef0c241f29"},
+    "combine": {"bytes": 506731776, "src_sha": "829d3f12a04df5c7"},
+    "dispatch_fp8": {"bytes": 242761728, "src_sha": "438eeea93673c608"},
+    "layout+dispatch_fp8": {"bytes": 247802368, "src_sha": "f0b9cfcc2a1aba1c"},
+    "layout": {"bytes": 211712, "src_sha": "f0b9cfcc2a1aba1c"},
 }
 
 
