@@ -818,7 +818,8 @@ layout_count_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     zero_words(s.hr, R);
     __syncthreads();
     PairsT<CH> P;
-    const bool bad = load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
+    const bool bad =
+        load_and_rank<kRankKeys, CH>(idx, n, k, E_ids, key_div, E, blockIdx.x, tokens_per_block(k, CH), s, P);
     if (with_ranks) rank_sets<CH>(k, E, R, s, P);
     __syncthreads();
     warp_offsets(E, s);
@@ -966,9 +967,10 @@ layout_cluster_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, 
 // another block, so no cooperative launch, no workspace and no bounded wait.
 
 // Measured on B200 (graph of 20 back-to-back layouts, E = 256, R = 64, top-8):
-// 128 / 1024 / 2048 / 4096 tokens take 5.6 / 7.3 / 8.0 / 10.4 us this way
-// against 6.2 / 8.8 / 9.5 / 10.2 us with the exchange; at 6144 tokens the
-// blocks no longer fit on the GPU at once and it loses (18.9 against 12.1).
+// 1024 / 2048 / 4096 tokens take 6.7 / 7.5 / 9.9 us this way against
+// 8.8 / 9.5 / 10.2 us with the exchange; at 6144 tokens the blocks no longer
+// fit on the GPU at once and it loses (18.9 against 12.1).  Batches of at
+// most one token per SM take the one-CTA-per-token kernel instead.
 #ifndef CGL_REP_MAX_PAIRS
 #define CGL_REP_MAX_PAIRS 32768
 #endif
@@ -1250,8 +1252,8 @@ layout_rep_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, int 
     rep_scan<NT>(idx, n, k, E, R, (int64_t)blockIdx.x * T, vec != 0, s);
     __syncthreads();
     if (threadIdx.x < kThreads)
-        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                       max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, nullptr);
+        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank,
+                       expert_offset, max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, nullptr);
 }
 
 // Fused decode path: the layout and the FP8 dispatch of a small batch (at most
@@ -1532,8 +1534,9 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
 //      per receive row (and one per scale row), so the HBM writes of early
 //      tokens overlap the reads of later ones; warps 1-7 stage the CTA's last
 //      tokens.
-// At kernel start the TMA engine is also asked to bring the CTA's x rows into
-// L2 (one contiguous range), so that staging reads hit L2.
+// At kernel start the TMA engine is also asked to bring the CTA's own ids,
+// then its x rows (one contiguous range), into L2, so that the id scan and the
+// staging reads hit L2; the block's own ids are checked only after the scan.
 // No CTA waits on another.  It runs only when a CTA's whole share fits in
 // shared memory (at hidden 7168 up to 28 tokens per CTA, 4144 on 148 SMs).
 
@@ -1733,8 +1736,8 @@ layout_dispatch_fp8_kernel(const int32_t *__restrict__ idx, int64_t n, int k, in
     rep_scan<kLdThreads>(idx, n, k, E, R, t0, vec != 0, s);
     __syncthreads();
     if (threadIdx.x < kThreads) {
-        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank, expert_offset,
-                       max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
+        rep_finish<CH>(idx, n, k, E, R, cap, check_pairs<CH>(E, P), P, tokens_per_expert, tokens_per_rank, in_rank,
+                       expert_offset, max_count, dst_pos, recv_src, recv_rows, status, s, scan_tmp, s_dst);
         lsync();   // every row of the block is in s_dst
         if (threadIdx.x < 32) {
             for (int g = 0; g < ng; ++g) {
