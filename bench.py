@@ -396,6 +396,30 @@ class GpuStep:
         return calls
 
 
+def copy_probe(dev, nbytes: int = 1 << 30, reps: int = 10):
+    """HBM copy bandwidth of this device, read + write bytes (a device-to-device
+    tensor copy of nbytes, timed with CUDA events after two warm-up copies):
+    context for the roofline when no measured peak is on file."""
+    import torch
+
+    a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    b = torch.empty_like(a)
+    a.fill_(1)
+    for _ in range(2):
+        b.copy_(a)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(reps):
+        b.copy_(a)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    gbs = 2 * nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del a, b
+    torch.cuda.empty_cache()
+    return gbs
+
+
 def time_alone(step: GpuStep, reps: int, peak: float):
     """Each kernel of the step launched back to back: a CUDA graph of 20 launches
     (captured on a side stream after 3 eager warm-up launches) replayed until
@@ -434,8 +458,21 @@ def time_alone(step: GpuStep, reps: int, peak: float):
     return out
 
 
-def capture_step(step: GpuStep):
-    """One step's launches captured into a CUDA graph (on a side stream, after two eager runs)."""
+def graph_chunk(steps: int, cap: int = 20) -> int:
+    """Steps captured per CUDA graph in the timed passes: the largest divisor
+    of `steps` up to `cap`, so that exactly `steps` steps run.  Inside one graph
+    consecutive steps follow each other as launches of one stream do (each
+    kernel may start while the previous one drains); between two replays every
+    replay pays the graph launch, which at the decode shape is as long as a
+    kernel."""
+    for s in range(min(cap, steps), 0, -1):
+        if steps % s == 0:
+            return s
+    return 1
+
+
+def capture_step(step: GpuStep, nsteps: int = 1):
+    """`nsteps` steps' launches captured into one CUDA graph (on a side stream, after two eager runs)."""
     import torch
 
     torch.cuda.synchronize()
@@ -448,7 +485,8 @@ def capture_step(step: GpuStep):
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        step.run()
+        for _ in range(nsteps):
+            step.run()
     torch.cuda.synchronize()
     return g
 
@@ -456,10 +494,10 @@ def capture_step(step: GpuStep):
 def time_phase_graphs(step: GpuStep, steps: int):
     """Per-phase step time without events between kernels.
 
-    The combine phase alone: a CUDA graph holding only the step's combine
-    launch, replayed `steps` times between two events (its input, the expert
-    outputs, is larger than L2, so back-to-back replays read HBM like the step
-    does).  The dispatch phase (layout + dispatch) is the rest of the clean
+    The combine phase alone: a CUDA graph holding graph_chunk(steps) of the
+    step's combine launches, replayed to `steps` launches between two events
+    (its input, the expert outputs, is larger than L2, so back-to-back
+    launches read HBM like the step does).  The dispatch phase (layout + dispatch) is the rest of the clean
     step: ms_per_step minus that.  Timing the dispatch phase the same way would
     flatter it, because its input x (56 MiB at the prefill shape) stays in L2
     between back-to-back replays, while in the step the combine evicts it."""
@@ -478,15 +516,17 @@ def time_phase_graphs(step: GpuStep, steps: int):
             call()
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    chunk = graph_chunk(steps)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        call()
+        for _ in range(chunk):
+            call()
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(steps):
+    for _ in range(steps // chunk):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
@@ -697,7 +737,9 @@ def run_ours(args):
                    fused_decode=args.fused_decode, split_layout=args.split_layout, pow2_scales=args.ue8m0)
     phases = step.kernels()
 
-    graph = None if args.no_graph else capture_step(step)
+    chunk = graph_chunk(args.steps)
+    graph = None if args.no_graph else capture_step(step)                  # one step: the warm-up
+    graph_k = None if args.no_graph else capture_step(step, chunk)         # `chunk` steps: the timed pass
     for _ in range(args.warmup):
         if graph is not None:
             graph.replay()
@@ -712,13 +754,13 @@ def run_ours(args):
         time.sleep(0.3)   # let nvidia-smi start sampling before the timed region
     # timed region: K steps, one event on each side, nothing between the kernels
     # (an event between two kernels stops the next one from launching early);
-    # by default each step is one replay of a CUDA graph holding the step's launches
+    # by default K / chunk replays of a CUDA graph holding `chunk` steps' launches
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record()
-    if graph is not None:
-        for _ in range(args.steps):
-            graph.replay()
+    if graph_k is not None:
+        for _ in range(args.steps // chunk):
+            graph_k.replay()
     else:
         for _ in range(args.steps):
             step.run()
@@ -791,12 +833,18 @@ def run_ours(args):
                                  "to about min(K, 200) launches between two CUDA events, after 3 warm-up launches"),
 
         "gpu_launches": args.steps * sum(p[1] for p in phases),
-        "launch": "eager" if args.no_graph else "CUDA graph of one step, replayed K times (e2e and per-kernel passes eager)",
+        "launch": "eager" if args.no_graph else (f"CUDA graph of {chunk} steps, replayed K/{chunk} times (warm-up: a "
+                                                 "one-step graph; e2e and per-kernel passes eager)"),
         "kernel_timing": ("per-kernel us from a second pass of the same K steps with a CUDA event "
                           f"after every kernel ({ms_instr * 1e3:.1f} us/step there vs {ms * 1e3:.1f} clean); "
                           "each includes the launch gap the events add"),
         "clocks": clocks, "device_status": status_bits or "ok",
     })
+    if peak_src != "measured":   # no measured peak on file: the same kind of copy, measured here
+        probe = copy_probe(dev)
+        line["hbm_copy_probe"] = {"gbs": probe, "dominant_frac_of_probe": roof["achieved"] / probe,
+                                  "how": "device-to-device copy of 1 GiB, read + write bytes, CUDA events, "
+                                         "after the timed passes"}
     if ms_comb is not None:
         nb = {n: b for n, _, b in phases}
         comb_b = nb.get("combine", 0)
@@ -804,8 +852,9 @@ def run_ours(args):
             "dispatch_us": (ms - ms_comb) * 1e3, "combine_us": ms_comb * 1e3,
             "dispatch_gbs": (step.step_bytes() - comb_b) / ((ms - ms_comb) * 1e-3) / 1e9,
             "combine_gbs": comb_b / (ms_comb * 1e-3) / 1e9,
-            "phase_timing": ("no event between kernels: combine_us = a CUDA graph of the step's combine launch "
-                             "alone, replayed K times (its expert-output input exceeds L2); dispatch_us = "
+            "phase_timing": ("no event between kernels: combine_us = the step's combine launch alone, K launches "
+                             "from a CUDA graph of the same chunk of launches as the step's (its expert-output "
+                             "input exceeds L2); dispatch_us = "
                              "ms_per_step - combine_us (layout and dispatch, with the transitions of the step); "
                              "the instrumented per-kernel split is under 'kernels'"),
         })
