@@ -1352,6 +1352,13 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     const int nd = G > 1 ? rep_designated(b, G, R) : 0;
     const uint32_t rm = div_magic(E / R), gm = div_magic(G);
     griddep_wait();   // ids and x may come from the kernels just before
+    // the dispatch's first pass over the CTA's token: its x loads are in flight
+    // through the layout (16 values per thread)
+    uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+    if (kDispatch && has_tok && tid < (h >> 4)) {
+        xa = ld_nc_v4(x + t * h + (int64_t)tid * 16);
+        xb = ld_nc_v4(x + t * h + (int64_t)tid * 16 + 8);
+    }
     // this thread's token (n <= 256 = the block size): its ids, in flight while zeroing
     int32_t ids[KM];
     const int64_t tp = tid;
@@ -1491,8 +1498,8 @@ decode_token_kernel(const int32_t *__restrict__ idx, int64_t n, int k, int E, in
     for (int c0 = warp * 32; c0 < chunks; c0 += NT) {   // warp-uniform
         const int c = c0 + lane;
         const bool active = c < chunks;
-        uint4 a = make_uint4(0, 0, 0, 0), bb = a;
-        if (active) {
+        uint4 a = xa, bb = xb;   // the first pass was loaded at the start (c == tid)
+        if (c0 != warp * 32 && active) {
             a = ld_nc_v4(x + t * h + (int64_t)c * 16);
             bb = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
         }
