@@ -45,8 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {
     "combine": {"bytes": 506731776, "src_sha": "829d3f12a04df5c7"},
     "dispatch_fp8": {"bytes": 242761728, "src_sha": "438eeea93673c608"},
-    "layout+dispatch_fp8": {"bytes": 247802368, "src_sha": "f0b9cfcc2a1aba1c"},
-    "layout": {"bytes": 211712, "src_sha": "f0b9cfcc2a1aba1c"},
+    "layout+dispatch_fp8": {"bytes": 249300224, "src_sha": "fc8c8394cdf9dd22"},
+    "layout": {"bytes": 212480, "src_sha": "fc8c8394cdf9dd22"},
 }
 
 
