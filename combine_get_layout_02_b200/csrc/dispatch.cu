@@ -39,8 +39,10 @@ constexpr int kMaxBulkHiddenBf16 = 8192; // two staged BF16 rows stay within 32 
 __global__ void __launch_bounds__(1024)
 dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                          const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
-                         float *__restrict__ recv_scale, int64_t recv_rows, int pow2, uint32_t *status) {
+                         float *__restrict__ recv_scale, int64_t recv_rows, int pow2,
+                         unsigned long long *claim, uint32_t *status) {
     extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][h] staged code rows
+    __shared__ int64_t s_next[2];      // claimed tokens (dynamic order)
     griddep_wait();                   // dst_pos (and x) may come from the kernels just before
     const int chunks = h >> 4, nblk = h >> 7;
     const int c = threadIdx.x;        // this thread's 16 values
@@ -48,15 +50,29 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
     const bool scale_lane = active && (c & 7) == 0;
     bool bad = false;
     int buf = 0;
-    int64_t t = blockIdx.x;
+    // Token order.  Static: CTA b takes tokens b, b + G, ...  Dynamic (claim
+    // != null, a counter that is zero at launch): thread 0 claims the CTA's
+    // tokens from the counter, one token ahead of the one being loaded, so CTAs
+    // on SMs that stream faster take more tokens (on B200 some SMs, by where
+    // they sit, are consistently slower).
+    int64_t t = blockIdx.x, tn = t + gridDim.x, pend = n;
+    if (claim != nullptr) {
+        if (threadIdx.x == 0) {
+            s_next[0] = (int64_t)atomicAdd(claim, 1ull);
+            s_next[1] = (int64_t)atomicAdd(claim, 1ull);
+        }
+        __syncthreads();
+        t = s_next[0];
+        tn = t < n ? s_next[1] : n;
+        if (threadIdx.x == 0 && tn < n) pend = (int64_t)atomicAdd(claim, 1ull);
+    }
     uint4 a = make_uint4(0, 0, 0, 0), b = a;
     if (t < n && active) {
         a = ld_nc_v4(x + t * h + (int64_t)c * 16);
         b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
     }
-    for (; t < n; t += gridDim.x, buf ^= 1) {
-        const int64_t tn = t + gridDim.x;   // prefetch the next token's chunk
-        uint4 an = make_uint4(0, 0, 0, 0), bn = an;
+    for (int it = 0; t < n; buf ^= 1, ++it) {
+        uint4 an = make_uint4(0, 0, 0, 0), bn = an;   // the next token's chunk, in flight
         if (tn < n && active) {
             an = ld_nc_v4(x + tn * h + (int64_t)c * 16);
             bn = ld_nc_v4(x + tn * h + (int64_t)c * 16 + 8);
@@ -70,11 +86,19 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         block_scale(amax_c, pow2 != 0, scale, inv);
         const uint4 q = quant16(a, b, inv);
         uint8_t *row = rows_smem + buf * h;
-        if (threadIdx.x == 0) bulk_wait_read<1>();   // copies from two tokens ago have read `row`
+        if (threadIdx.x == 0) {
+            bulk_wait_read<1>();   // copies from two tokens ago have read `row`
+            if (claim != nullptr) s_next[it & 1] = pend < n ? pend : n;
+        }
         __syncthreads();
         if (active) *reinterpret_cast<uint4 *>(row + c * 16) = q;
         fence_proxy_async();
         __syncthreads();
+        int64_t tnn = tn + gridDim.x;   // the token after the next one
+        if (claim != nullptr) {
+            tnn = tn < n ? s_next[it & 1] : n;
+            if (threadIdx.x == 0) pend = tnn < n ? (int64_t)atomicAdd(claim, 1ull) : n;
+        }
         const int32_t *dp = dst_pos + t * k;
         if (threadIdx.x == 0) {
             for (int j = 0; j < k; ++j) {
@@ -93,6 +117,8 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         }
         a = an;
         b = bn;
+        t = tn;
+        tn = tnn;
     }
     if (threadIdx.x == 0) bulk_wait_all();
     if (bad) report(status, kErrRange);
@@ -242,7 +268,8 @@ dispatch_bf16_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
 
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
-                               int num_sms, bool pow2, uint32_t *status, cudaStream_t stream) {
+                               int num_sms, bool pow2, uint32_t *status, cudaStream_t stream,
+                               unsigned long long *claim) {
     if (n * (h / 16) == 0) return CGL_OK;
     if (h <= kMaxBulkHidden) {
         const int threads = (h / 16 + 31) / 32 * 32;
@@ -251,7 +278,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
         if (grid <= 0) return CGL_ECUDA;
         const cudaError_t err = launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)2 * h, stream, x, n, h, k, dst_pos, recv_x,
-                                           recv_scale, recv_rows, (int)pow2, status);
+                                           recv_scale, recv_rows, (int)pow2, claim, status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
     }
     const int64_t work = n * (h / 16);

@@ -2001,8 +2001,13 @@ cgl_status launch_token_kernel(const int32_t *idx, int64_t n, int k, int E, int 
 
 size_t layout_workspace_bytes(int64_t n, int k, int E, int R) { return ws_layout(n, k, E, R).bytes; }
 
+// Workspace of cgl_layout_dispatch_fp8: the layout's, then (16-byte aligned) a
+// 64-bit token counter for the dispatch kernel when the layout and the
+// dispatch run as two kernels; the fused kernel needs none.
+size_t ld_claim_offset(int64_t n, int k, int E, int R) { return align16(ws_layout(n, k, E, R).bytes); }
+
 size_t layout_dispatch_workspace_bytes(int64_t n, int k, int E, int R) {
-    return ws_layout(n, k, E, R).bytes;   // the fused kernel needs none; the split path the layout's
+    return ld_claim_offset(n, k, E, R) + 16;
 }
 
 bool layout_dispatch_fused_fits(int64_t n, int k, int E, int R, int h, int num_sms) {
@@ -2047,11 +2052,18 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
                                     stream);
         }
     }
+    // two kernels: the dispatch hands its tokens out from a counter at the
+    // workspace's tail, zeroed here first (before the layout, so that nothing
+    // comes between the two kernels)
+    unsigned long long *claim =
+        reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + ld_claim_offset(n, k, E, R));
+    if (cudaMemsetAsync(claim, 0, sizeof(unsigned long long), stream) != cudaSuccess) return CGL_ECUDA;
     const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
                                         expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
     if (st != CGL_OK) return st;
     const int64_t recv_rows = cap > 0 ? (int64_t)E * cap : n * k;
-    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, num_sms, pow2, status, stream);
+    return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, num_sms, pow2, status, stream,
+                               claim);
 }
 
 bool layout_needs_smem_optin(int E, int R, int k) {

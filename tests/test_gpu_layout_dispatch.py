@@ -140,3 +140,49 @@ def test_layout_dispatch_fp8_graph_replays(oracle_mod):
         assert np.array_equal(rx.cpu().numpy()[used], ox[used])
         assert np.array_equal(rs.cpu().numpy()[used].view(np.uint32), os_[used].view(np.uint32))
     del g
+
+
+@pytest.mark.parametrize("num_tokens,num_sms", [(6000, 0), (16384, 0), (5000, 37)])
+def test_layout_dispatch_fp8_two_kernels_hand_tokens_out_dynamically(oracle_mod, num_tokens, num_sms):
+    """Past the fused kernel's range the call runs the layout and then the
+    dispatch kernel, whose CTAs claim tokens from a counter at the workspace's
+    tail (zeroed by the call).  Every token is dispatched exactly once, bit for
+    bit, whatever the workspace held before (the counter word included), call
+    after call on one workspace and in graph replays."""
+    inp = W.make_inputs("skewed", 3, num_tokens=num_tokens)
+    wl = inp.workload
+    E, R = wl.num_experts, wl.num_ranks
+    n, k = inp.topk_idx.shape
+    assert cgl.layout_dispatch_kernel_count(n, k, E, R, wl.hidden, num_sms=num_sms) > 1
+    nbytes = cgl.layout_dispatch_workspace_bytes(n, k, E, R)
+    ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device=dev())   # counter word far from zero
+    idx, x = i32(inp.topk_idx), to_bf16(inp.x)
+    L = oracle_mod.get_layout(inp.topk_idx, E, R)
+    ox, os_ = oracle_mod.dispatch_fp8(inp.x, L.dst_pos, n * k)
+    used = L.recv_src >= 0
+
+    def check(rx, rs, st):
+        assert np.array_equal(rx.cpu().numpy()[used], ox[used]), "codes"
+        assert np.array_equal(rs.cpu().numpy()[used].view(np.uint32), os_[used].view(np.uint32)), "scales"
+        assert st.item() == 0
+
+    rx = torch.full((n * k, wl.hidden), 0x5A, dtype=torch.uint8, device=dev())
+    rs = torch.full((n * k, wl.hidden // 128), -2.0, dtype=torch.float32, device=dev())
+    st = cgl.new_status(dev())
+    for _ in range(3):
+        lay, rx, rs = cgl.layout_dispatch_fp8(idx, x, E, R, recv_x=rx, recv_scale=rs, workspace=ws, status=st,
+                                              num_sms=num_sms)
+        torch.cuda.synchronize()
+        assert np.array_equal(lay.dst_pos.cpu().numpy(), L.dst_pos)
+        check(rx, rs, st)
+        rx.fill_(0x5A)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cgl.layout_dispatch_fp8(idx, x, E, R, out=lay, recv_x=rx, recv_scale=rs, workspace=ws, status=st,
+                                num_sms=num_sms)
+    for _ in range(2):
+        rx.fill_(0x5A)
+        g.replay()
+        torch.cuda.synchronize()
+        check(rx, rs, st)
+    del g
