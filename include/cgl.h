@@ -315,8 +315,8 @@ cgl_status cgl_decode_dispatch_fp8(const int32_t *topk_idx, int64_t num_tokens, 
 
 /*
  * Bytes of device workspace cgl_layout_dispatch_fp8 needs for these sizes
- * (per-block counts for up to 256 blocks, or cgl_get_layout's workspace when
- * that is larger).  Host-only; 0 for invalid sizes.
+ * (cgl_get_layout's workspace, then, 16-byte aligned, the dispatch kernel's
+ * token counter).  Host-only; 0 for invalid sizes.
  */
 size_t cgl_layout_dispatch_workspace_bytes(int64_t num_tokens, int num_topk, int num_experts, int num_ranks);
 
@@ -334,16 +334,20 @@ int cgl_layout_dispatch_kernel_count(int64_t num_tokens, int num_topk, int num_e
  * cgl_get_layout, FP8 dispatch as for cgl_dispatch_fp8 (brainleap "Day2
  * DeepEP": the normal kernels' prefill setting, FP8 dispatch with BF16
  * combine).  The pages have no fused form; on one GPU it lets the FP8
- * dispatch's reads and quantisation run while the layout's blocks exchange
- * their counts.
+ * dispatch's reads and quantisation run while the layout's counts are made.
  * Same outputs, ordering and errors as cgl_get_layout followed by
  * cgl_dispatch_fp8 with the layout's dst_pos (receive rows = E*capacity when
  * opts.capacity > 0, else num_tokens*num_topk).
- * One cooperative kernel (one CTA of 768 threads per SM, each owning
- * ceil(num_tokens / SMs) tokens) when every SM gets at least 64 (token, slot)
- * pairs, num_experts % 8 == 0 and a CTA's whole share of FP8 rows fits in shared memory (at hidden
- * 7168: up to 28 tokens per CTA, 4144 tokens on 148 SMs); otherwise the
- * layout kernel(s) then the dispatch kernel, with the same results.
+ * One kernel when it applies: one CTA per token when there is at most one
+ * token per SM in use (decode); for prefill-sized batches (every SM gets at
+ * least 64 (token, slot) pairs, at most 32768 pairs, and a CTA's whole share
+ * of FP8 rows fits in shared memory: at hidden 7168 up to 28 tokens per CTA,
+ * 4144 tokens on 148 SMs) one CTA of 768 threads per SM, each owning
+ * ceil(num_tokens / SMs) tokens, which reads every id for the counts (no CTA
+ * waits on another) while it stages its tokens' FP8 rows.  Otherwise the
+ * layout kernel(s), then the dispatch kernel, whose CTAs take their tokens
+ * from a counter at the workspace's tail that the call zeroes first (CTAs
+ * on faster SMs take more); the same results either way.
  * opts.num_sms caps the SMs used.
  * workspace: device, >= cgl_layout_dispatch_workspace_bytes(...) bytes,
  *   16-byte aligned, any contents (scratch for the call; overlapping calls
