@@ -43,10 +43,10 @@ FALLBACK_HBM_GBS = 6650.0
 # source and the shared device header it was taken on; a changed source
 # reports traffic null.
 NCU_TRAFFIC = {
-    "combine": {"bytes": 506731776, "src_sha": "829d3f12a04df5c7"},
-    "dispatch_fp8": {"bytes": 242761728, "src_sha": "438eeea93673c608"},
-    "layout+dispatch_fp8": {"bytes": 249300224, "src_sha": "fc8c8394cdf9dd22"},
-    "layout": {"bytes": 212480, "src_sha": "fc8c8394cdf9dd22"},
+    "combine": {"bytes": 508535552, "src_sha": "829d3f12a04df5c7"},
+    "dispatch_fp8": {"bytes": 242461952, "src_sha": "be18baca93105f91"},
+    "layout+dispatch_fp8": {"bytes": 247885568, "src_sha": "56936daaa2c37330"},
+    "layout": {"bytes": 212480, "src_sha": "56936daaa2c37330"},
 }
 
 
