@@ -36,3 +36,15 @@ def test_warmup_below_three_is_refused():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
                        capture_output=True, text=True, timeout=120, env=env, cwd=ROOT)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_graph_chunk_times_exactly_k_steps():
+    # the timed pass replays a graph of `chunk` steps K / chunk times: chunk divides K, at most 20
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for k in (1, 2, 3, 7, 20, 21, 40, 97, 200, 300, 2000, 2001):
+        c = bench.graph_chunk(k)
+        assert 1 <= c <= 20 and k % c == 0, (k, c)
+        assert all(k % d for d in range(c + 1, min(k, 20) + 1)), (k, c)   # the largest such divisor
+    assert bench.graph_chunk(2000) == 20 and bench.graph_chunk(97) == 1 and bench.graph_chunk(3) == 3
