@@ -2,7 +2,8 @@
 """Benchmark of the MoE layout -> FP8 dispatch -> BF16 combine path on B200.
 
 One step = cgl_get_layout + cgl_dispatch_fp8 + cgl_combine over one batch of
-synthetic routing (the 4096-token prefill shape by default: hidden 7168, 256
+synthetic routing (batches of at most one token per SM: cgl_layout_dispatch_fp8,
+one launch, + cgl_combine) (the 4096-token prefill shape by default: hidden 7168, 256
 experts in 8 groups, top-4 groups / top-8 experts, 64 logical ranks) with all
 inputs resident in HBM.  The metric is the step's algorithmic HBM bytes per
 second; per-kernel microseconds and fractions of the measured HBM peak are in
@@ -186,7 +187,8 @@ class GpuStep:
     """Device buffers for one workload and the launch sequence of one step."""
 
     def __init__(self, wl: W.Workload, seed: int, device, dedup: bool = False, full_backward: bool = False,
-                 fused_decode: bool = False, split_layout: bool = False, pow2_scales: bool = False):
+                 fused_decode: bool = False, split_layout: bool = False, pow2_scales: bool = False,
+                 fused_layout: bool = False):
         import torch
 
         import combine_get_layout_02_b200 as cgl
@@ -196,9 +198,15 @@ class GpuStep:
         self.pow2 = pow2_scales
         self.full_backward = full_backward and wl.with_grad and not dedup
         self.fused_decode = fused_decode and wl.fp8 and not dedup
-        # FP8 steps call cgl_layout_dispatch_fp8 (one cooperative kernel when it
-        # applies, else the layout and dispatch kernels) unless asked to split
-        self.layout_dispatch = wl.fp8 and not dedup and not self.fused_decode and not split_layout
+        # FP8 steps: the library's three calls (cgl_get_layout, cgl_dispatch_fp8
+        # handing tokens out from a scratch counter, cgl_combine), measured a
+        # little faster at prefill than the fused cgl_layout_dispatch_fp8 kernel;
+        # batches of at most one token per SM take cgl_layout_dispatch_fp8 (one
+        # launch, one CTA per token).  --fused-layout: cgl_layout_dispatch_fp8
+        # at every size; --split-layout: the three calls at every size.
+        one_per_sm = wl.num_tokens <= torch.cuda.get_device_properties(device).multi_processor_count
+        self.layout_dispatch = (wl.fp8 and not dedup and not self.fused_decode and not split_layout
+                                and (fused_layout or one_per_sm))
         inp = W.make_inputs(wl, seed)
         n, h, k = wl.num_tokens, wl.hidden, wl.topk
         self.host = inp
@@ -215,6 +223,8 @@ class GpuStep:
         self.y = bf16(y_host).to(device)
         self.grad = bf16(inp.grad).to(device) if inp.grad is not None else None
         self.status = cgl.new_status(device)
+        # the standalone dispatch calls hand tokens out from a counter in this scratch (cgl_opts.scratch)
+        self.scratch = cgl.new_scratch(device)
         E, R = wl.num_experts, wl.num_ranks
         self.ws = torch.empty(max(cgl.layout_workspace_bytes(n, k, E, R),
                                   cgl.layout_dispatch_workspace_bytes(n, k, E, R)), dtype=torch.uint8, device=device)
@@ -320,26 +330,28 @@ class GpuStep:
             rec()
             if wl.fp8:
                 cgl.dispatch_fp8(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
-                                 recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2)
+                                 recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2,
+                                 scratch=self.scratch)
             else:
                 cgl.dispatch_bf16(self.x, self.rlay.rank_dst, self.rrows, recv_x=self.recv_x,
-                                  status=self.status)
+                                  status=self.status, scratch=self.scratch)
             rec()
             cgl.combine(self.y, self.rlay.rank_dst, self.w_rank, out=self.out, status=self.status)
             rec()
             if wl.with_grad:
                 cgl.dispatch_bf16(self.grad, self.rlay.rank_dst, self.rrows, recv_x=self.grad_recv,
-                                  status=self.status)
+                                  status=self.status, scratch=self.scratch)
                 rec()
             return
         cgl.get_layout(self.idx, E, R, self.cap, workspace=self.ws, out=self.lay, status=self.status)
         rec()
         if wl.fp8:
             cgl.dispatch_fp8(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
-                             recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2)
+                             recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2,
+                             scratch=self.scratch)
         else:
             cgl.dispatch_bf16(self.x, self.lay.dst_pos, self.rows, recv_x=self.recv_x,
-                              status=self.status)
+                              status=self.status, scratch=self.scratch)
         rec()
         cgl.combine(self.y, self.lay.dst_pos, self.w, out=self.out, status=self.status)
         rec()
@@ -349,7 +361,7 @@ class GpuStep:
                                      grad_w=self.grad_w, status=self.status)
             else:
                 cgl.dispatch_bf16(self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv,
-                                  status=self.status)
+                                  status=self.status, scratch=self.scratch)
             rec()
 
     def _event(self):
@@ -372,7 +384,8 @@ class GpuStep:
         calls = [("layout", lay_call, b["layout"])]
         if wl.fp8:
             calls.append(("dispatch_fp8", lambda: cgl.dispatch_fp8(self.x, dst, rows, recv_x=self.recv_x,
-                                                                   recv_scale=self.recv_scale, status=self.status, pow2_scales=self.pow2),
+                                                                   recv_scale=self.recv_scale, status=self.status,
+                                                                   pow2_scales=self.pow2, scratch=self.scratch),
                           b["dispatch_fp8"]))
             if self.layout_dispatch:
                 calls.append(("layout+dispatch_fp8", lambda: cgl.layout_dispatch_fp8(
@@ -380,7 +393,8 @@ class GpuStep:
                     workspace=self.ws, status=self.status, pow2_scales=self.pow2), b["layout"] + b["dispatch_fp8"]))
         else:
             calls.append(("dispatch_bf16", lambda: cgl.dispatch_bf16(self.x, dst, rows, recv_x=self.recv_x,
-                                                                     status=self.status), b["dispatch_bf16"]))
+                                                                     status=self.status, scratch=self.scratch),
+                          b["dispatch_bf16"]))
         calls.append(("combine", lambda: cgl.combine(self.y, dst, w, out=self.out, status=self.status),
                       b["combine"]))
         if wl.with_grad and not self.dedup:
@@ -391,8 +405,8 @@ class GpuStep:
                     status=self.status), 2 * n * h + 4 * n * k * h + 12 * n * k))
             else:
                 calls.append(("combine_backward", lambda: cgl.dispatch_bf16(
-                    self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv, status=self.status),
-                    b["dispatch_bf16"]))
+                    self.grad, self.lay.dst_pos, self.rows, recv_x=self.grad_recv, status=self.status,
+                    scratch=self.scratch), b["dispatch_bf16"]))
         return calls
 
 
@@ -547,6 +561,7 @@ def _twin(step: GpuStep) -> GpuStep:
         if isinstance(v, torch.Tensor):
             setattr(t, name, torch.empty_like(v))
     t.status = step.cgl.new_status(step.dev)
+    t.scratch = step.cgl.new_scratch(step.dev)
     for name in ("lay", "rlay"):
         v = getattr(step, name, None)
         if v is not None:
@@ -734,7 +749,8 @@ def run_ours(args):
 
         wl = dataclasses.replace(wl, num_tokens=args.num_tokens)
     step = GpuStep(wl, rank_seed(args.seed, rank), dev, dedup=args.dedup, full_backward=args.full_backward,
-                   fused_decode=args.fused_decode, split_layout=args.split_layout, pow2_scales=args.ue8m0)
+                   fused_decode=args.fused_decode, split_layout=args.split_layout, pow2_scales=args.ue8m0,
+                   fused_layout=args.fused_layout)
     phases = step.kernels()
 
     chunk = graph_chunk(args.steps)
@@ -896,7 +912,10 @@ def main(argv=None):
     ap.add_argument("--fused-decode", action="store_true",
                     help="layout and FP8 dispatch in one launch (batches of at most 1024 token-slot pairs)")
     ap.add_argument("--split-layout", action="store_true",
-                    help="FP8: cgl_get_layout and cgl_dispatch_fp8 as two calls instead of cgl_layout_dispatch_fp8")
+                    help="FP8: cgl_get_layout and cgl_dispatch_fp8 as two calls at every size (the default above "
+                         "one token per SM)")
+    ap.add_argument("--fused-layout", action="store_true",
+                    help="FP8: cgl_layout_dispatch_fp8 at every size (at prefill sizes one fused kernel)")
     ap.add_argument("--no-graph", action="store_true", help="launch each timed step eagerly instead of replaying a CUDA graph")
     ap.add_argument("--ue8m0", action="store_true", help="FP8: power-of-two (UE8M0) scales instead of amax / 448")
     args = ap.parse_args(argv)

@@ -48,7 +48,7 @@ class CglError(RuntimeError):
 
 
 class Opts(C.Structure):
-    _fields_ = [("num_sms", C.c_int32), ("capacity", C.c_int32), ("flags", C.c_uint32)]
+    _fields_ = [("num_sms", C.c_int32), ("capacity", C.c_int32), ("flags", C.c_uint32), ("scratch", C.c_void_p)]
 
 
 OPT_UE8M0_SCALES = 1   # cgl_opts.flags: power-of-two (UE8M0) FP8 scales
@@ -134,8 +134,20 @@ def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None):
     return t
 
 
-def _opts(num_sms: int = 0, capacity: int = 0, pow2_scales: bool = False):
-    return C.byref(Opts(int(num_sms), int(capacity), OPT_UE8M0_SCALES if pow2_scales else 0))
+def _opts(num_sms: int = 0, capacity: int = 0, pow2_scales: bool = False, scratch: Optional[torch.Tensor] = None):
+    sp = None
+    if scratch is not None:
+        if not scratch.is_cuda or scratch.numel() * scratch.element_size() < 16 or not scratch.is_contiguous():
+            raise CglError(EINVAL, "scratch", "a contiguous device tensor of at least 16 bytes")
+        sp = scratch.data_ptr()
+    return C.byref(Opts(int(num_sms), int(capacity), OPT_UE8M0_SCALES if pow2_scales else 0, sp))
+
+
+def new_scratch(device=None) -> torch.Tensor:
+    """Zeroed 16-byte device scratch (cgl_opts.scratch) for dispatch_fp8 / dispatch_bf16: with it the
+    dispatch kernel hands tokens out dynamically; each call leaves it zero.  Calls that may run at the
+    same time need their own."""
+    return torch.zeros(2, dtype=torch.int64, device=device or "cuda")
 
 
 def new_status(device=None) -> torch.Tensor:
@@ -252,10 +264,12 @@ def get_rank_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, ca
 
 def dispatch_fp8(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
                  recv_x: Optional[torch.Tensor] = None, recv_scale: Optional[torch.Tensor] = None,
-                 status: Optional[torch.Tensor] = None, num_sms: int = 0, pow2_scales: bool = False, stream=None):
+                 status: Optional[torch.Tensor] = None, num_sms: int = 0, pow2_scales: bool = False,
+                 scratch: Optional[torch.Tensor] = None, stream=None):
     """FP8 E4M3 dispatch with per-token 1x128 fp32 scales (cgl_dispatch_fp8).
 
     pow2_scales: power-of-two (UE8M0) scales (CGL_OPT_UE8M0_SCALES).
+    scratch: new_scratch() (cgl_opts.scratch): tokens handed out dynamically, same results.
     Returns (recv_x uint8 [rows, H], recv_scale fp32 [rows, H/128]); rows that
     receive no copy are left as they were (uninitialised when allocated here)."""
     x = _dev(x, "x", torch.bfloat16, 2)
@@ -267,15 +281,18 @@ def dispatch_fp8(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
     if recv_scale is None:
         recv_scale = torch.empty((num_recv_rows, h // 128), dtype=torch.float32, device=x.device)
     code = lib().cgl_dispatch_fp8(_ptr(x), n, h, k, _ptr(dst), _ptr(recv_x), _ptr(recv_scale),
-                                  int(num_recv_rows), _opts(num_sms, 0, pow2_scales), _ptr(status), _stream(stream))
+                                  int(num_recv_rows), _opts(num_sms, 0, pow2_scales, scratch), _ptr(status),
+                                  _stream(stream))
     _check(code, "cgl_dispatch_fp8")
     return recv_x, recv_scale
 
 
 def dispatch_bf16(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
                   recv_x: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
-                  num_sms: int = 0, stream=None) -> torch.Tensor:
-    """BF16 row dispatch (cgl_dispatch_bf16); also the combine-backward re-dispatch of grads."""
+                  num_sms: int = 0, scratch: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """BF16 row dispatch (cgl_dispatch_bf16); also the combine-backward re-dispatch of grads.
+
+    scratch: new_scratch() (cgl_opts.scratch): tokens handed out dynamically, same results."""
     x = _dev(x, "x", torch.bfloat16, 2)
     dst = _dev(dst_pos, "dst_pos", torch.int32, 2)
     n, h = x.shape
@@ -283,7 +300,7 @@ def dispatch_bf16(x: torch.Tensor, dst_pos: torch.Tensor, num_recv_rows: int, *,
     if recv_x is None:
         recv_x = torch.empty((num_recv_rows, h), dtype=torch.bfloat16, device=x.device)
     code = lib().cgl_dispatch_bf16(_ptr(x), n, h, k, _ptr(dst), _ptr(recv_x), int(num_recv_rows),
-                                   _opts(num_sms), _ptr(status), _stream(stream))
+                                   _opts(num_sms, 0, False, scratch), _ptr(status), _stream(stream))
     _check(code, "cgl_dispatch_bf16")
     return recv_x
 

@@ -35,6 +35,9 @@ int opt_cap(const cgl_opts *o) { return o ? o->capacity : 0; }
 uint32_t opt_flags(const cgl_opts *o) { return o ? o->flags : 0u; }
 bool flags_ok(const cgl_opts *o) { return (opt_flags(o) & ~CGL_OPT_UE8M0_SCALES) == 0; }
 bool opt_pow2(const cgl_opts *o) { return (opt_flags(o) & CGL_OPT_UE8M0_SCALES) != 0; }
+unsigned long long *opt_scratch(const cgl_opts *o) {
+    return o ? static_cast<unsigned long long *>(o->scratch) : nullptr;
+}
 
 }  // namespace
 
@@ -128,7 +131,7 @@ using namespace cgl;
 
 extern "C" {
 
-int cgl_version(void) { return 200; }
+int cgl_version(void) { return 300; }
 
 const char *cgl_status_string(int s) {
     switch (s) {
@@ -214,10 +217,10 @@ cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const in
     if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && (!recv_x || !recv_scale)) return CGL_EINVAL;
     if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) ||
-        !aligned(recv_scale, 4) || !aligned(status_dev, 4))
+        !aligned(recv_scale, 4) || !aligned(status_dev, 4) || !aligned(opt_scratch(opts), 8))
         return CGL_EALIGN;
     return launch_dispatch_fp8(x, n, h, k, dst_pos, recv_x, recv_scale, recv_rows, opt_sms(opts), opt_pow2(opts),
-                               status_dev, static_cast<cudaStream_t>(stream));
+                               status_dev, static_cast<cudaStream_t>(stream), opt_scratch(opts));
 }
 
 cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
@@ -227,10 +230,11 @@ cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const i
     if (opt_sms(opts) < 0 || !flags_ok(opts)) return CGL_EINVAL;
     if (n > 0 && (!x || !dst_pos)) return CGL_EINVAL;
     if (n > 0 && recv_rows > 0 && !recv_x) return CGL_EINVAL;
-    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) || !aligned(status_dev, 4))
+    if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(dst_pos, 4) || !aligned(status_dev, 4) ||
+        !aligned(opt_scratch(opts), 8))
         return CGL_EALIGN;
     return launch_dispatch_bf16(x, n, h, k, dst_pos, recv_x, recv_rows, opt_sms(opts), status_dev,
-                                static_cast<cudaStream_t>(stream));
+                                static_cast<cudaStream_t>(stream), opt_scratch(opts));
 }
 
 cgl_status cgl_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_pos,

@@ -51,10 +51,10 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
     bool bad = false;
     int buf = 0;
     // Token order.  Static: CTA b takes tokens b, b + G, ...  Dynamic (claim
-    // != null, a counter that is zero at launch): thread 0 claims the CTA's
-    // tokens from the counter, one token ahead of the one being loaded, so CTAs
-    // on SMs that stream faster take more tokens (on B200 some SMs, by where
-    // they sit, are consistently slower).
+    // != null: a token counter and a finished-CTA count, both zero at launch):
+    // thread 0 claims the CTA's tokens from the counter, one token ahead of the
+    // one being loaded, so CTAs on SMs that stream faster take more tokens (on
+    // B200 some SMs, by where they sit, are consistently slower).
     int64_t t = blockIdx.x, tn = t + gridDim.x, pend = n;
     if (claim != nullptr) {
         if (threadIdx.x == 0) {
@@ -120,7 +120,14 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         t = tn;
         tn = tnn;
     }
-    if (threadIdx.x == 0) bulk_wait_all();
+    if (threadIdx.x == 0) {
+        bulk_wait_all();
+        // the last CTA to finish leaves the counter words zero for the next launch
+        if (claim != nullptr && atomicAdd(claim + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+            claim[0] = 0;
+            claim[1] = 0;
+        }
+    }
     if (bad) report(status, kErrRange);
 }
 
@@ -192,8 +199,9 @@ dispatch_fp8_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
 __global__ void __launch_bounds__(1024)
 dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                           const int32_t *__restrict__ dst_pos, uint16_t *__restrict__ recv_x,
-                          int64_t recv_rows, uint32_t *status) {
+                          int64_t recv_rows, unsigned long long *claim, uint32_t *status) {
     extern __shared__ __align__(128) uint8_t rows_smem[];   // [2][2h] staged rows
+    __shared__ int64_t s_next[2];      // claimed tokens (dynamic order, as in the FP8 kernel)
     griddep_wait();
     const int chunks = h >> 4;
     const int c = threadIdx.x;
@@ -201,21 +209,33 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
     const uint32_t row_bytes = (uint32_t)h * 2;
     bool bad = false;
     int buf = 0;
-    int64_t t = blockIdx.x;
+    int64_t t = blockIdx.x, tn = t + gridDim.x, pend = n;
+    if (claim != nullptr) {
+        if (threadIdx.x == 0) {
+            s_next[0] = (int64_t)atomicAdd(claim, 1ull);
+            s_next[1] = (int64_t)atomicAdd(claim, 1ull);
+        }
+        __syncthreads();
+        t = s_next[0];
+        tn = t < n ? s_next[1] : n;
+        if (threadIdx.x == 0 && tn < n) pend = (int64_t)atomicAdd(claim, 1ull);
+    }
     uint4 a = make_uint4(0, 0, 0, 0), b = a;
     if (t < n && active) {
         a = ld_nc_v4(x + t * h + (int64_t)c * 16);
         b = ld_nc_v4(x + t * h + (int64_t)c * 16 + 8);
     }
-    for (; t < n; t += gridDim.x, buf ^= 1) {
-        const int64_t tn = t + gridDim.x;
-        uint4 an = make_uint4(0, 0, 0, 0), bn = an;
+    for (int it = 0; t < n; buf ^= 1, ++it) {
+        uint4 an = make_uint4(0, 0, 0, 0), bn = an;   // the next token's chunk, in flight
         if (tn < n && active) {
             an = ld_nc_v4(x + tn * h + (int64_t)c * 16);
             bn = ld_nc_v4(x + tn * h + (int64_t)c * 16 + 8);
         }
         uint8_t *row = rows_smem + (size_t)buf * row_bytes;
-        if (threadIdx.x == 0) bulk_wait_read<1>();
+        if (threadIdx.x == 0) {
+            bulk_wait_read<1>();
+            if (claim != nullptr) s_next[it & 1] = pend < n ? pend : n;
+        }
         __syncthreads();
         if (active) {
             reinterpret_cast<uint4 *>(row)[2 * c] = a;
@@ -223,6 +243,11 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
         }
         fence_proxy_async();
         __syncthreads();
+        int64_t tnn = tn + gridDim.x;   // the token after the next one
+        if (claim != nullptr) {
+            tnn = tn < n ? s_next[it & 1] : n;
+            if (threadIdx.x == 0) pend = tnn < n ? (int64_t)atomicAdd(claim, 1ull) : n;
+        }
         if (threadIdx.x == 0) {
             const int32_t *dp = dst_pos + t * k;
             for (int j = 0; j < k; ++j) {
@@ -235,8 +260,16 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
         }
         a = an;
         b = bn;
+        t = tn;
+        tn = tnn;
     }
-    if (threadIdx.x == 0) bulk_wait_all();
+    if (threadIdx.x == 0) {
+        bulk_wait_all();
+        if (claim != nullptr && atomicAdd(claim + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+            claim[0] = 0;
+            claim[1] = 0;
+        }
+    }
     if (bad) report(status, kErrRange);
 }
 
@@ -292,7 +325,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
 
 cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                 uint16_t *recv_x, int64_t recv_rows, int num_sms, uint32_t *status,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, unsigned long long *claim) {
     if (n * (h / 8) == 0) return CGL_OK;
     if (h % 16 == 0 && h <= kMaxBulkHiddenBf16) {
         const int threads = (h / 16 + 31) / 32 * 32;
@@ -301,7 +334,7 @@ cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, cons
         if (grid <= 0) return CGL_ECUDA;
         const cudaError_t err = launch_pdl(dispatch_bf16_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)4 * h, stream, x, n, h, k, dst_pos, recv_x,
-                                           recv_rows, status);
+                                           recv_rows, claim, status);
         return err == cudaSuccess ? CGL_OK : CGL_ECUDA;
     }
     const int64_t work = n * (h / 8);

@@ -64,8 +64,9 @@ cgl_status launch_rank_layout(const int32_t *idx, int64_t n, int k, int E, int R
                               cudaStream_t stream);
 
 // pow2: power-of-two (UE8M0) scales instead of amax_c / 448 (cgl_opts.flags).
-// claim: null (static token order), or a 64-bit counter that is zero when the
-// kernel starts, from which the CTAs claim tokens (dynamic order).
+// claim: null (static token order), or two 64-bit words that are zero when
+// the kernel starts (a token counter the CTAs claim from, and a count of
+// finished CTAs); the last CTA to finish zeroes both again.
 cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                uint8_t *recv_x, float *recv_scale, int64_t recv_rows,
                                int num_sms, bool pow2, uint32_t *status, cudaStream_t stream,
@@ -73,7 +74,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
 
 cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, const int32_t *dst_pos,
                                 uint16_t *recv_x, int64_t recv_rows, int num_sms, uint32_t *status,
-                                cudaStream_t stream);
+                                cudaStream_t stream, unsigned long long *claim = nullptr);
 
 cgl_status launch_combine(const uint16_t *y, int64_t recv_rows, const int32_t *dst_pos,
                           const float *w, int64_t n, int h, int k, uint16_t *out, int num_sms,

@@ -2057,7 +2057,7 @@ cgl_status launch_layout_dispatch_fp8(const int32_t *idx, int64_t n, int k, int 
     // comes between the two kernels)
     unsigned long long *claim =
         reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + ld_claim_offset(n, k, E, R));
-    if (cudaMemsetAsync(claim, 0, sizeof(unsigned long long), stream) != cudaSuccess) return CGL_ECUDA;
+    if (cudaMemsetAsync(claim, 0, 2 * sizeof(unsigned long long), stream) != cudaSuccess) return CGL_ECUDA;
     const cgl_status st = launch_layout(idx, n, k, E, R, cap, tokens_per_expert, tokens_per_rank, in_rank,
                                         expert_offset, max_count, dst_pos, recv_src, ws, status, stream);
     if (st != CGL_OK) return st;

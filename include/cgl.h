@@ -88,12 +88,23 @@ typedef struct cgl_opts {
      * values: 2^e, whose biased exponent field ((bits >> 23) & 0xFF) is the
      * UE8M0 code.  Calls that quantise nothing ignore the flag. */
     uint32_t flags;
+    /* Optional device scratch for cgl_dispatch_fp8 and cgl_dispatch_bf16: 16
+     * bytes, 8-byte aligned, all zero before the first call that uses them.
+     * With it the dispatch kernel's CTAs claim their tokens from a counter in
+     * it instead of taking a fixed share (on B200 some SMs, by where they sit,
+     * stream measurably slower; the faster ones then take more tokens), with
+     * results identical to the fixed order; the kernel leaves the 16 bytes
+     * zero again when it finishes.  Calls that may run at the same time must
+     * not share one scratch (stream-ordered calls may).  NULL: fixed order.
+     * Other calls ignore it. */
+    void *scratch;
 } cgl_opts;
 
 #define CGL_OPT_UE8M0_SCALES 1u
 
 /* Library version (major * 10000 + minor * 100 + patch).  0.2.0 added
- * cgl_opts.flags: C callers built against an older cgl.h must be rebuilt. */
+ * cgl_opts.flags and 0.3.0 cgl_opts.scratch: C callers built against an older
+ * cgl.h must be rebuilt. */
 int cgl_version(void);
 
 /* A static string naming a cgl_status value (or "unknown status"). */
@@ -248,6 +259,8 @@ cgl_status cgl_get_layout_noalloc(const int32_t *topk_idx, int64_t num_tokens, i
  *   [num_recv_rows, hidden/128].  Rows that receive no copy are NOT written.
  * Requires hidden % 128 == 0; x and recv_x 16-byte aligned; dst_pos and
  * recv_scale 4-byte aligned.
+ * With opts->scratch the CTAs claim tokens dynamically (see cgl_opts.scratch);
+ * the results are the same.
  * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows (that copy is skipped).
  */
 cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t num_tokens, int hidden, int num_topk,
@@ -262,7 +275,8 @@ cgl_status cgl_dispatch_fp8(const uint16_t *x, int64_t num_tokens, int hidden, i
  * combine format of the benchmark settings.
  * In (device): x BF16 [num_tokens, hidden]; dst_pos int32 [num_tokens, num_topk].
  * Out (device): recv_x BF16 [num_recv_rows, hidden]; rows with no copy are not written.
- * Requires hidden % 8 == 0; x and recv_x 16-byte aligned.
+ * Requires hidden % 8 == 0; x and recv_x 16-byte aligned.  With opts->scratch
+ * (hidden % 16 == 0 and <= 8192) the CTAs claim tokens dynamically.
  * Device errors: CGL_ERANGE if some dst_pos >= num_recv_rows.
  */
 cgl_status cgl_dispatch_bf16(const uint16_t *x, int64_t num_tokens, int hidden, int num_topk,

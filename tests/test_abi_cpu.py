@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import combine_get_layout_02_b200 as cgl
 from combine_get_layout_02_b200 import build as cbuild
@@ -236,3 +237,19 @@ def test_opts_flags_unknown_bits_refused(L):
     # the defined bit passes the flag check (then fails on a misaligned pointer, as without it)
     ok = C.byref(cgl.Opts(0, 0, cgl.OPT_UE8M0_SCALES))
     assert L.cgl_dispatch_fp8(p + 8, 128, 7168, 8, p, p, p, 1024, ok, p, None) == cgl.EALIGN
+
+
+def test_opts_scratch_alignment_and_layout(L):
+    """cgl_opts.scratch (library 0.3.0): a device pointer after flags; the dispatch
+    calls refuse one that is not 8-byte aligned before launching anything (fake
+    pointers never used); NULL keeps the fixed token order."""
+    src = open(os.path.join(ROOT, "include", "cgl.h")).read()
+    assert "void *scratch;" in src and L.cgl_version() >= 300
+    assert [f[0] for f in cgl.Opts._fields_] == ["num_sms", "capacity", "flags", "scratch"]
+    assert C.sizeof(cgl.Opts) == 24 and cgl.Opts.scratch.offset == 16
+    p = FAKE
+    mis = C.byref(cgl.Opts(0, 0, 0, p + 4))
+    assert L.cgl_dispatch_fp8(p, 128, 7168, 8, p, p, p, 1024, mis, p, None) == cgl.EALIGN
+    assert L.cgl_dispatch_bf16(p, 128, 7168, 8, p, p, 1024, mis, p, None) == cgl.EALIGN
+    with pytest.raises(cgl.CglError):
+        cgl._opts(scratch=torch.zeros(2, dtype=torch.int64))          # a host tensor is refused

@@ -142,3 +142,71 @@ def test_bf16_dispatch_and_backward_full_size(oracle_mod, name):
         assert np.array_equal(bits(g), oracle_mod.dispatch_bf16(inp.grad, L.dst_pos, rows))
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("name,num_sms", [("prefill", 0), ("skewed", 0), ("decode", 0), ("prefill", 23)])
+def test_fp8_dispatch_with_scratch_hands_tokens_out(oracle_mod, name, num_sms):
+    """cgl_opts.scratch: the dispatch CTAs claim tokens from a counter in it.
+    Same bytes and scales as the oracle (and the fixed order), call after call
+    on one scratch, which every call leaves zero; in a graph replay too."""
+    inp = W.make_inputs(name, 0)
+    wl = inp.workload
+    E, R = wl.num_experts, wl.num_ranks
+    cap = oracle_mod.get_layout(inp.topk_idx, E, R).max_count if wl.padded else 0
+    lay = cgl.get_layout(i32(inp.topk_idx), E, R, cap)
+    rows = lay.num_recv_rows
+    L = oracle_mod.get_layout(inp.topk_idx, E, R, cap)
+    ox, os_ = oracle_mod.dispatch_fp8(inp.x, L.dst_pos, rows)
+    used = L.recv_src >= 0
+    x = to_bf16(inp.x)
+    sc = cgl.new_scratch(dev())
+    st = cgl.new_status(dev())
+    rx = torch.zeros((rows, wl.hidden), dtype=torch.uint8, device=dev())
+    rs = torch.zeros((rows, wl.hidden // 128), dtype=torch.float32, device=dev())
+
+    def check():
+        torch.cuda.synchronize()
+        assert np.array_equal(rx.cpu().numpy()[used], ox[used])
+        assert np.array_equal(rs.cpu().numpy()[used].view(np.uint32), os_[used].view(np.uint32))
+        assert int(st.item()) == 0 and torch.count_nonzero(sc).item() == 0
+
+    for _ in range(3):
+        rx.zero_()
+        cgl.dispatch_fp8(x, lay.dst_pos, rows, recv_x=rx, recv_scale=rs, status=st, num_sms=num_sms, scratch=sc)
+        check()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cgl.dispatch_fp8(x, lay.dst_pos, rows, recv_x=rx, recv_scale=rs, status=st, num_sms=num_sms, scratch=sc)
+    for _ in range(2):
+        rx.zero_()
+        g.replay()
+        check()
+    del g
+
+
+def test_bf16_dispatch_with_scratch_hands_tokens_out(oracle_mod):
+    """cgl_opts.scratch on the BF16 dispatch (and the combine-backward re-dispatch):
+    bit-exact rows at the BF16 workload's full size, scratch left zero; the
+    flattened kernel (hidden above the staged path's limit) ignores it."""
+    inp = W.make_inputs("bf16", 0)
+    wl = inp.workload
+    lay = cgl.get_layout(i32(inp.topk_idx), wl.num_experts, wl.num_ranks)
+    rows = lay.num_recv_rows
+    L = oracle_mod.get_layout(inp.topk_idx, wl.num_experts, wl.num_ranks)
+    sc = cgl.new_scratch(dev())
+    st = cgl.new_status(dev())
+    for src in (inp.x, inp.grad, inp.x):
+        recv = cgl.dispatch_bf16(to_bf16(src), lay.dst_pos, rows, status=st, scratch=sc)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(recv), oracle_mod.dispatch_bf16(src, L.dst_pos, rows))
+        assert torch.count_nonzero(sc).item() == 0
+    rng = np.random.default_rng(13)
+    n, h, k, E = 40, 9000, 3, 6
+    x = W.f32_to_bf16_bits(rng.standard_normal((n, h)).astype(np.float32))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(n)]).astype(np.int32)
+    lay2 = cgl.get_layout(i32(idx), E, 1)
+    got = cgl.dispatch_bf16(to_bf16(x), lay2.dst_pos, lay2.num_recv_rows, status=st, scratch=sc)
+    torch.cuda.synchronize()
+    L2 = oracle_mod.get_layout(idx, E, 1)
+    assert np.array_equal(bits(got), oracle_mod.dispatch_bf16(x, L2.dst_pos, lay2.num_recv_rows))
+    assert int(st.item()) == 0 and torch.count_nonzero(sc).item() == 0
