@@ -44,10 +44,10 @@ FALLBACK_HBM_GBS = 6650.0
 # source and the shared device header it was taken on; a changed source
 # reports traffic null.
 NCU_TRAFFIC = {
-    "combine": {"bytes": 508535552, "src_sha": "829d3f12a04df5c7"},
-    "dispatch_fp8": {"bytes": 242461952, "src_sha": "be18baca93105f91"},
-    "layout+dispatch_fp8": {"bytes": 247885568, "src_sha": "56936daaa2c37330"},
-    "layout": {"bytes": 212480, "src_sha": "56936daaa2c37330"},
+    "combine": {"bytes": 507279104, "src_sha": "829d3f12a04df5c7"},
+    "dispatch_fp8": {"bytes": 242931712, "src_sha": "2144efd6d31fdbf7"},
+    "layout+dispatch_fp8": {"bytes": 247476480, "src_sha": "ff4c3e2d259d9d86"},
+    "layout": {"bytes": 212736, "src_sha": "ff4c3e2d259d9d86"},
 }
 
 

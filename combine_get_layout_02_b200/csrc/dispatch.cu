@@ -309,6 +309,7 @@ cgl_status launch_dispatch_fp8(const uint16_t *x, int64_t n, int h, int k, const
         const int grid = persistent_grid((const void *)dispatch_fp8_bulk_kernel, threads, (size_t)2 * h,
                                          kBulkThreadsPerSM / threads, num_sms, n);
         if (grid <= 0) return CGL_ECUDA;
+        if (n <= grid) claim = nullptr;   // one token per CTA either way: the counter would only add latency
         const cudaError_t err = launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)2 * h, stream, x, n, h, k, dst_pos, recv_x,
                                            recv_scale, recv_rows, (int)pow2, claim, status);
@@ -332,6 +333,7 @@ cgl_status launch_dispatch_bf16(const uint16_t *x, int64_t n, int h, int k, cons
         const int grid = persistent_grid((const void *)dispatch_bf16_bulk_kernel, threads, (size_t)4 * h,
                                          kBulkThreadsPerSM / threads, num_sms, n);
         if (grid <= 0) return CGL_ECUDA;
+        if (n <= grid) claim = nullptr;   // one token per CTA either way
         const cudaError_t err = launch_pdl(dispatch_bf16_bulk_kernel, dim3(grid), dim3(threads),
                                            (size_t)4 * h, stream, x, n, h, k, dst_pos, recv_x,
                                            recv_rows, claim, status);

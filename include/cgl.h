@@ -94,9 +94,10 @@ typedef struct cgl_opts {
      * it instead of taking a fixed share (on B200 some SMs, by where they sit,
      * stream measurably slower; the faster ones then take more tokens), with
      * results identical to the fixed order; the kernel leaves the 16 bytes
-     * zero again when it finishes.  Calls that may run at the same time must
-     * not share one scratch (stream-ordered calls may).  NULL: fixed order.
-     * Other calls ignore it. */
+     * zero again when it finishes (batches with at most one token per CTA
+     * keep the fixed order and leave it untouched).  Calls that may run at
+     * the same time must not share one scratch (stream-ordered calls may).
+     * NULL: fixed order.  Other calls ignore it. */
     void *scratch;
 } cgl_opts;
 
