@@ -17,7 +17,8 @@
 // global, each one whole 7168-byte receive row at hidden 7168, so the copies
 // leave the SM as long contiguous writes without holding registers.  Before a
 // buffer is rewritten, the copies issued from it two tokens earlier must have
-// read it (bulk wait_group.read).  The block leaders store the fp32 scales.
+// read it (bulk wait_group.read).  One lane of each 128-value block stores its
+// fp32 scale.
 //
 // BF16, hidden <= 8192 and a multiple of 16: the same staging with BF16 rows.
 // FP8 above 16384 and BF16 otherwise: one thread per 16 or 8 values of the
@@ -36,6 +37,33 @@ constexpr int kMaxBulkHidden = 16384;    // one thread per 16 values: at most 10
 constexpr int kBulkThreadsPerSM = 1024;  // CTAs per SM of the bulk kernels = this / block size
 constexpr int kMaxBulkHiddenBf16 = 8192; // two staged BF16 rows stay within 32 KiB of shared memory
 
+// Dynamic token order: thread 0 of each CTA claims tokens from a 64-bit word,
+// one ahead of the token being loaded.  Bits 0-39 count the tokens handed out,
+// bits 40-63 the CTAs that have finished: claims and counts are atomics on the
+// one word, so its modification order holds every CTA's claims before that
+// CTA's count, and the CTA whose count completes the grid can set the word
+// back to zero for the next launch with no fence.  A claim's raw value is only
+// looked at where it is used (take_claim), so the atomic's round trip overlaps
+// the token's copies.  take_claim clamps it to n: a word that did not start at
+// zero can at worst leave tokens out, never send a load or a copy outside the
+// batch.  A launch that starts from zero hands out at most n + 2 G tokens (no
+// CTA makes more than two claims past n); a claim of n + 3 G or more means the
+// scratch was not zero, and sets `bad` (reported as kErrRange).
+constexpr int kDoneShift = 40;
+constexpr unsigned long long kClaimMask = (1ull << kDoneShift) - 1;
+
+__device__ __forceinline__ int64_t take_claim(unsigned long long word, int64_t n, bool &bad) {
+    const unsigned long long v = word & kClaimMask;
+    if (v >= (unsigned long long)n + 3ull * gridDim.x) bad = true;
+    return v < (unsigned long long)n ? (int64_t)v : n;
+}
+
+// After the CTA's last claim: count it finished; the last CTA resets the word.
+__device__ __forceinline__ void claims_done(unsigned long long *claim) {
+    const unsigned long long old = atomicAdd(claim, 1ull << kDoneShift);
+    if ((old >> kDoneShift) == (unsigned long long)gridDim.x - 1) *claim = 0;
+}
+
 __global__ void __launch_bounds__(1024)
 dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k,
                          const int32_t *__restrict__ dst_pos, uint8_t *__restrict__ recv_x,
@@ -51,20 +79,21 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
     bool bad = false;
     int buf = 0;
     // Token order.  Static: CTA b takes tokens b, b + G, ...  Dynamic (claim
-    // != null: a token counter and a finished-CTA count, both zero at launch):
-    // thread 0 claims the CTA's tokens from the counter, one token ahead of the
+    // != null: the claim word above, zero at launch): thread 0 claims the
+    // CTA's tokens from the counter, one token ahead of the
     // one being loaded, so CTAs on SMs that stream faster take more tokens (on
     // B200 some SMs, by where they sit, are consistently slower).
-    int64_t t = blockIdx.x, tn = t + gridDim.x, pend = n;
+    int64_t t = blockIdx.x, tn = t + gridDim.x;
+    unsigned long long pend = (unsigned long long)n;   // thread 0: the claim in flight (raw)
     if (claim != nullptr) {
         if (threadIdx.x == 0) {
-            s_next[0] = (int64_t)atomicAdd(claim, 1ull);
-            s_next[1] = (int64_t)atomicAdd(claim, 1ull);
+            s_next[0] = take_claim(atomicAdd(claim, 1ull), n, bad);
+            s_next[1] = take_claim(atomicAdd(claim, 1ull), n, bad);
         }
         __syncthreads();
         t = s_next[0];
         tn = t < n ? s_next[1] : n;
-        if (threadIdx.x == 0 && tn < n) pend = (int64_t)atomicAdd(claim, 1ull);
+        if (threadIdx.x == 0 && tn < n) pend = atomicAdd(claim, 1ull);
     }
     uint4 a = make_uint4(0, 0, 0, 0), b = a;
     if (t < n && active) {
@@ -88,7 +117,7 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         uint8_t *row = rows_smem + buf * h;
         if (threadIdx.x == 0) {
             bulk_wait_read<1>();   // copies from two tokens ago have read `row`
-            if (claim != nullptr) s_next[it & 1] = pend < n ? pend : n;
+            if (claim != nullptr) s_next[it & 1] = take_claim(pend, n, bad);
         }
         __syncthreads();
         if (active) *reinterpret_cast<uint4 *>(row + c * 16) = q;
@@ -97,7 +126,7 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         int64_t tnn = tn + gridDim.x;   // the token after the next one
         if (claim != nullptr) {
             tnn = tn < n ? s_next[it & 1] : n;
-            if (threadIdx.x == 0) pend = tnn < n ? (int64_t)atomicAdd(claim, 1ull) : n;
+            if (threadIdx.x == 0) pend = tnn < n ? atomicAdd(claim, 1ull) : (unsigned long long)n;
         }
         const int32_t *dp = dst_pos + t * k;
         if (threadIdx.x == 0) {
@@ -121,12 +150,8 @@ dispatch_fp8_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int k
         tn = tnn;
     }
     if (threadIdx.x == 0) {
+        if (claim != nullptr) claims_done(claim);   // before the wait, which hides the atomic
         bulk_wait_all();
-        // the last CTA to finish leaves the counter words zero for the next launch
-        if (claim != nullptr && atomicAdd(claim + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
-            claim[0] = 0;
-            claim[1] = 0;
-        }
     }
     if (bad) report(status, kErrRange);
 }
@@ -209,16 +234,17 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
     const uint32_t row_bytes = (uint32_t)h * 2;
     bool bad = false;
     int buf = 0;
-    int64_t t = blockIdx.x, tn = t + gridDim.x, pend = n;
+    int64_t t = blockIdx.x, tn = t + gridDim.x;
+    unsigned long long pend = (unsigned long long)n;   // thread 0: the claim in flight (raw)
     if (claim != nullptr) {
         if (threadIdx.x == 0) {
-            s_next[0] = (int64_t)atomicAdd(claim, 1ull);
-            s_next[1] = (int64_t)atomicAdd(claim, 1ull);
+            s_next[0] = take_claim(atomicAdd(claim, 1ull), n, bad);
+            s_next[1] = take_claim(atomicAdd(claim, 1ull), n, bad);
         }
         __syncthreads();
         t = s_next[0];
         tn = t < n ? s_next[1] : n;
-        if (threadIdx.x == 0 && tn < n) pend = (int64_t)atomicAdd(claim, 1ull);
+        if (threadIdx.x == 0 && tn < n) pend = atomicAdd(claim, 1ull);
     }
     uint4 a = make_uint4(0, 0, 0, 0), b = a;
     if (t < n && active) {
@@ -234,7 +260,7 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
         uint8_t *row = rows_smem + (size_t)buf * row_bytes;
         if (threadIdx.x == 0) {
             bulk_wait_read<1>();
-            if (claim != nullptr) s_next[it & 1] = pend < n ? pend : n;
+            if (claim != nullptr) s_next[it & 1] = take_claim(pend, n, bad);
         }
         __syncthreads();
         if (active) {
@@ -246,7 +272,7 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
         int64_t tnn = tn + gridDim.x;   // the token after the next one
         if (claim != nullptr) {
             tnn = tn < n ? s_next[it & 1] : n;
-            if (threadIdx.x == 0) pend = tnn < n ? (int64_t)atomicAdd(claim, 1ull) : n;
+            if (threadIdx.x == 0) pend = tnn < n ? atomicAdd(claim, 1ull) : (unsigned long long)n;
         }
         if (threadIdx.x == 0) {
             const int32_t *dp = dst_pos + t * k;
@@ -264,11 +290,8 @@ dispatch_bf16_bulk_kernel(const uint16_t *__restrict__ x, int64_t n, int h, int 
         tn = tnn;
     }
     if (threadIdx.x == 0) {
+        if (claim != nullptr) claims_done(claim);   // before the wait, which hides the atomic
         bulk_wait_all();
-        if (claim != nullptr && atomicAdd(claim + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
-            claim[0] = 0;
-            claim[1] = 0;
-        }
     }
     if (bad) report(status, kErrRange);
 }

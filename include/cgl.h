@@ -96,7 +96,13 @@ typedef struct cgl_opts {
      * results identical to the fixed order; the kernel leaves the 16 bytes
      * zero again when it finishes (batches with at most one token per CTA
      * keep the fixed order and leave it untouched).  Calls that may run at
-     * the same time must not share one scratch (stream-ordered calls may).
+     * the same time must not share one scratch (stream-ordered calls may),
+     * and the scratch must stay allocated as long as a captured CUDA graph
+     * that uses it may be replayed.  A scratch that was not zero cannot make
+     * the kernel touch memory outside the call's buffers (claims past the
+     * batch are clamped), but tokens may be left out: when a claim returns a
+     * value that no zeroed start produces (>= num_tokens + 3 * CTAs), the
+     * kernel sets the CGL_ERANGE bit in *status.
      * NULL: fixed order.  Other calls ignore it. */
     void *scratch;
 } cgl_opts;

@@ -210,3 +210,43 @@ def test_bf16_dispatch_with_scratch_hands_tokens_out(oracle_mod):
     L2 = oracle_mod.get_layout(idx, E, 1)
     assert np.array_equal(bits(got), oracle_mod.dispatch_bf16(x, L2.dst_pos, lay2.num_recv_rows))
     assert int(st.item()) == 0 and torch.count_nonzero(sc).item() == 0
+
+
+@pytest.mark.parametrize("start", [10**9, -1])
+def test_dispatch_scratch_not_zero_is_reported(oracle_mod, start):
+    """A scratch whose counter did not start at zero (here 1e9, or 2^64 - 1 as
+    the int64 -1) is clamped by the kernel: every claim past the batch becomes
+    "no token", nothing outside the buffers is touched, and CGL_ERANGE is set.
+    The launch still leaves the scratch zero, so the next call is exact."""
+    inp = W.make_inputs("prefill", 0)
+    wl = inp.workload
+    lay = cgl.get_layout(i32(inp.topk_idx), wl.num_experts, wl.num_ranks)
+    rows = lay.num_recv_rows
+    L = oracle_mod.get_layout(inp.topk_idx, wl.num_experts, wl.num_ranks)
+    ox, os_ = oracle_mod.dispatch_fp8(inp.x, L.dst_pos, rows)
+    x = to_bf16(inp.x)
+    rx = torch.zeros((rows, wl.hidden), dtype=torch.uint8, device=dev())
+    rs = torch.zeros((rows, wl.hidden // 128), dtype=torch.float32, device=dev())
+    for kind in ("fp8", "bf16"):
+        sc = torch.tensor([start, 0], dtype=torch.int64, device=dev())
+        st = cgl.new_status(dev())
+        if kind == "fp8":
+            cgl.dispatch_fp8(x, lay.dst_pos, rows, recv_x=rx, recv_scale=rs, status=st, scratch=sc)
+        else:
+            cgl.dispatch_bf16(x, lay.dst_pos, rows, status=st, scratch=sc)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 1 << cgl.ERANGE
+        assert torch.count_nonzero(sc).item() == 0
+        st.zero_()
+        rx.zero_()
+        if kind == "fp8":
+            cgl.dispatch_fp8(x, lay.dst_pos, rows, recv_x=rx, recv_scale=rs, status=st, scratch=sc)
+            torch.cuda.synchronize()
+            used = L.recv_src >= 0
+            assert np.array_equal(rx.cpu().numpy()[used], ox[used])
+            assert np.array_equal(rs.cpu().numpy()[used].view(np.uint32), os_[used].view(np.uint32))
+        else:
+            got = cgl.dispatch_bf16(x, lay.dst_pos, rows, status=st, scratch=sc)
+            torch.cuda.synchronize()
+            assert np.array_equal(bits(got), oracle_mod.dispatch_bf16(inp.x, L.dst_pos, rows))
+        assert int(st.item()) == 0
