@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # reports traffic null.
 NCU_TRAFFIC = {
     "combine": {"bytes": 507279104, "src_sha": "829d3f12a04df5c7"},
-    "dispatch_fp8": {"bytes": 242931712, "src_sha": "2144efd6d31fdbf7"},
+    "dispatch_fp8": {"bytes": 243865088, "src_sha": "1e399167ee854d42"},
     "layout+dispatch_fp8": {"bytes": 247476480, "src_sha": "ff4c3e2d259d9d86"},
     "layout": {"bytes": 212736, "src_sha": "ff4c3e2d259d9d86"},
 }
