@@ -182,6 +182,17 @@ def test_fp8_dispatch_with_scratch_hands_tokens_out(oracle_mod, name, num_sms):
         g.replay()
         check()
     del g
+    # stream-ordered calls may share one scratch: FP8 and BF16 dispatches back to
+    # back with no host synchronisation between them, each starting from the word
+    # the one before left zero
+    rx.zero_()
+    check_bf16 = wl.hidden <= 8192 and rows * wl.hidden <= 1 << 28   # host copies stay under 1 GB
+    for _ in range(3):
+        cgl.dispatch_fp8(x, lay.dst_pos, rows, recv_x=rx, recv_scale=rs, status=st, num_sms=num_sms, scratch=sc)
+        rb = cgl.dispatch_bf16(x, lay.dst_pos, rows, status=st, num_sms=num_sms, scratch=sc)
+    check()
+    if check_bf16:
+        assert np.array_equal(bits(rb)[used], oracle_mod.dispatch_bf16(inp.x, L.dst_pos, rows)[used])
 
 
 def test_bf16_dispatch_with_scratch_hands_tokens_out(oracle_mod):
